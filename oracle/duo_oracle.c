@@ -1,0 +1,180 @@
+/*
+ * Plain fp64 CPU oracle for mixed-head (DuoAttention) attention.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg load this file's library. It shares no code, header, table
+ * or helper with the CUDA path in mixed_head_kv_b200/.
+ *
+ * What it computes (DuoAttention abstract, "read the original abstract" on the
+ * pith.science review page; restated on the sourcepulse project card, "How It
+ * Works"): every attention head is either
+ *   - a retrieval head, which keeps a full KV cache and attends to every
+ *     previous token, or
+ *   - a streaming head, which keeps a constant-length cache holding the
+ *     attention-sink tokens and the most recent tokens, and attends only to
+ *     those.
+ * For GQA models the head type belongs to the KV head and every query head of
+ * its group inherits it.
+ *
+ * Readings of points the pages leave open (each is listed in the design doc):
+ *   - key set of a streaming head for a query at absolute position p:
+ *       K(p) = { j <= p : j < sink  or  p - j < recent }
+ *     ("recent" counts the query's own token; the union counts a key once);
+ *   - retrieval head: K(p) = { 0 .. p } (causal);
+ *   - scores s_j = scale * <q_p, k_j>, weights a_j = exp(s_j - max) / sum,
+ *     output o_p = sum_j a_j v_j, everything in double precision from bf16
+ *     inputs widened exactly;
+ *   - streaming cache slots: slot p for a sink position p < sink, ring slot
+ *     sink + (p - sink) mod recent otherwise (a fixed sink region plus a ring).
+ *
+ * All loops are the definitions written out: no blocking, no online softmax,
+ * no reordering beyond summation order.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* bf16 bit pattern -> double (exact: bf16 is the top half of an IEEE binary32). */
+static double bf16_to_double(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Membership of key position j in the key set of a query at position p.
+ * Retrieval head: every previous token. Streaming head: attention sinks plus
+ * the recent window (abstract: streaming heads "focus on recent tokens and
+ * attention sinks" with a constant-length cache). */
+int duo_oracle_key_allowed(int is_retrieval, int64_t p, int64_t j, int64_t sink, int64_t recent) {
+    if (j < 0 || j > p) return 0;
+    if (is_retrieval) return 1;
+    return (j < sink) || (p - j < recent);
+}
+
+/* Attention of one query row over an explicit list of key rows.
+ * q[D]; keys/vals: n rows of D bf16 each, row i at keys + i*D.
+ * out[D] receives sum_i a_i v_i; *wsum receives sum_i a_i (1 up to rounding).
+ * Returns 0, or -1 when the list is empty or allocation fails. */
+int duo_oracle_attend_rows(const uint16_t* q, const uint16_t* keys, const uint16_t* vals,
+                           int64_t n, int D, double scale, double* out, double* wsum) {
+    if (n <= 0) return -1;
+    double* s = (double*)malloc(sizeof(double) * (size_t)n);
+    if (!s) return -1;
+    double m = -INFINITY;
+    for (int64_t i = 0; i < n; ++i) {
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += bf16_to_double(q[d]) * bf16_to_double(keys[i * D + d]);
+        s[i] = scale * dot;
+        if (s[i] > m) m = s[i];
+    }
+    double denom = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        s[i] = exp(s[i] - m);
+        denom += s[i];
+    }
+    for (int d = 0; d < D; ++d) out[d] = 0.0;
+    double total = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        double a = s[i] / denom;
+        total += a;
+        for (int d = 0; d < D; ++d) out[d] += a * bf16_to_double(vals[i * D + d]);
+    }
+    if (wsum) *wsum = total;
+    free(s);
+    return 0;
+}
+
+/* Attention of one query at absolute position p of one head over the full
+ * key/value history of its KV head (k_hist/v_hist: T rows, row j = position j),
+ * restricted to the key set K(p) of that head's type. */
+static int attend_masked(const uint16_t* q, const uint16_t* k_hist, const uint16_t* v_hist,
+                         int64_t T, int D, int64_t p, int is_retrieval, int64_t sink,
+                         int64_t recent, double scale, double* out, double* wsum) {
+    int64_t last = p < T - 1 ? p : T - 1;
+    int64_t n = 0;
+    for (int64_t j = 0; j <= last; ++j) n += duo_oracle_key_allowed(is_retrieval, p, j, sink, recent);
+    if (n == 0) return -1;
+    uint16_t* kk = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * D));
+    uint16_t* vv = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * D));
+    if (!kk || !vv) { free(kk); free(vv); return -1; }
+    int64_t c = 0;
+    for (int64_t j = 0; j <= last; ++j) {
+        if (!duo_oracle_key_allowed(is_retrieval, p, j, sink, recent)) continue;
+        memcpy(kk + c * D, k_hist + j * D, sizeof(uint16_t) * (size_t)D);
+        memcpy(vv + c * D, v_hist + j * D, sizeof(uint16_t) * (size_t)D);
+        ++c;
+    }
+    int rc = duo_oracle_attend_rows(q, kk, vv, n, D, scale, out, wsum);
+    free(kk);
+    free(vv);
+    return rc;
+}
+
+/* Mixed-head attention for a batch of queries.
+ *   q      [B][Hq][NQ][D]   bf16 bits; query i of every head sits at position qpos[i]
+ *   k, v   [B][Hkv][T][D]   bf16 bits; row j is the token at position j
+ *   is_retrieval [Hkv]      1 = retrieval KV head, 0 = streaming KV head
+ *   out    [B][Hq][NQ][D]   double
+ *   wsum   [B][Hq][NQ]      double, optional: sum of the softmax weights
+ * Query head h reads KV head h / (Hq / Hkv). Returns the number of rows that
+ * failed (empty key set), 0 on success. Threads: OpenMP over (b, h, i). */
+int64_t duo_oracle_attention(const uint16_t* q, const int64_t* qpos, const uint16_t* k,
+                             const uint16_t* v, const uint8_t* is_retrieval, int B, int Hq,
+                             int Hkv, int64_t NQ, int64_t T, int D, int64_t sink, int64_t recent,
+                             double scale, double* out, double* wsum) {
+    int G = Hq / Hkv;
+    int64_t total = (int64_t)B * Hq * NQ;
+    int64_t failed = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : failed)
+    for (int64_t idx = 0; idx < total; ++idx) {
+        int64_t i = idx % NQ;
+        int h = (int)((idx / NQ) % Hq);
+        int b = (int)(idx / (NQ * Hq));
+        int g = h / G;
+        const uint16_t* qr = q + (((int64_t)b * Hq + h) * NQ + i) * D;
+        const uint16_t* kh = k + ((int64_t)b * Hkv + g) * T * D;
+        const uint16_t* vh = v + ((int64_t)b * Hkv + g) * T * D;
+        double ws = 0.0;
+        int rc = attend_masked(qr, kh, vh, T, D, qpos[i], is_retrieval[g], sink, recent, scale,
+                               out + idx * D, &ws);
+        if (wsum) wsum[idx] = ws;
+        if (rc != 0) failed += 1;
+    }
+    return failed;
+}
+
+/* Cache slot model: which absolute position each slot of one head's cache
+ * holds after `len` tokens were appended (closed form), -1 for an empty slot.
+ *   retrieval head: slot j holds position j for j < len;
+ *   streaming head (nslots = sink + recent): slot s < sink holds position s;
+ *     slot sink + r holds the latest position p < len with p >= sink and
+ *     (p - sink) mod recent == r. */
+void duo_oracle_slot_positions(int is_retrieval, int64_t sink, int64_t recent, int64_t len,
+                               int64_t nslots, int64_t* pos) {
+    for (int64_t s = 0; s < nslots; ++s) {
+        pos[s] = -1;
+        if (is_retrieval || s < sink) {
+            if (s < len) pos[s] = s;
+            continue;
+        }
+        int64_t r = s - sink;
+        if (r >= recent) continue;
+        int64_t best = -1;
+        for (int64_t p = sink + r; p < len; p += recent) best = p; /* latest writer wins */
+        pos[s] = best;
+    }
+}
+
+/* Threads the OpenMP runtime will use for duo_oracle_attention. */
+int duo_oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
