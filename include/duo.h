@@ -1,0 +1,184 @@
+/*
+ * duo.h — C ABI of libduo: mixed-head (DuoAttention) attention on B200 (sm_100a).
+ *
+ * The method (DuoAttention abstract, pith.science review page, "read the
+ * original abstract"; sourcepulse project card, "How It Works"): each KV head
+ * of each layer is either a retrieval head, which keeps a full KV cache and
+ * attends causally over every previous token, or a streaming head, which keeps
+ * a constant-length KV cache of the first `sink` tokens (attention sinks) plus
+ * the `recent` most recent tokens, and attends only to those. In GQA models
+ * every query head inherits the type of its KV head. The library covers the two
+ * phases the pages speed up (pre-filling, in chunks, and decoding) and the
+ * per-head cache append/eviction behind them.
+ *
+ * Conventions (all calls):
+ *  - Tensors are bf16, row-major, contiguous, in device memory owned by the
+ *    caller, 16-byte aligned (DUO_ERR_ALIGNMENT otherwise).
+ *      prefill q / out   [batch][n_tok][num_q_heads][head_dim]
+ *      prefill k / v     [batch][n_tok][num_kv_heads][head_dim]
+ *      decode  q / out   [batch][num_q_heads][head_dim]
+ *      decode  k / v     [batch][num_kv_heads][head_dim]
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is stream-ordered and asynchronous; host-side cache lengths are
+ *    updated when the call is enqueued. Calls on one cache must be issued on
+ *    one stream (or ordered by the caller): they share the cache's device state.
+ *  - Argument errors are reported before any launch and leave the cache
+ *    unchanged. DUO_ERR_CUDA reports a failed launch or CUDA call.
+ *  - Positions are absolute token indices within a sequence, starting at 0.
+ *    All sequences of a batch have the same length.
+ *  - Positional encodings are the caller's: q and k arrive already encoded and
+ *    cached tokens keep their original positions (no re-indexing).
+ *  - Softmax scale: layout.softmax_scale, or 1/sqrt(head_dim) when it is 0.
+ */
+#ifndef DUO_H_
+#define DUO_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DUO_API __attribute__((visibility("default")))
+#else
+#define DUO_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum duo_status {
+    DUO_OK = 0,
+    DUO_ERR_INVALID_ARG = 1, /* bad layout, mask, layer, size or null pointer */
+    DUO_ERR_CAPACITY = 2,    /* a retrieval cache would exceed max_len tokens */
+    DUO_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned */
+    DUO_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed */
+    DUO_ERR_STATE = 5,       /* call not valid in the cache's current state */
+    DUO_ERR_DEVICE = 6       /* a kernel reported a device-side error (see duo_cache_error) */
+} duo_status;
+
+/* Largest head counts the kernels accept. */
+#define DUO_MAX_Q_HEADS 256
+#define DUO_MAX_KV_HEADS 128
+
+/* Shape of the model's attention and of the caches.
+ *   num_layers    >= 1
+ *   batch         >= 1 sequences, all of the same length
+ *   num_q_heads   query heads, a multiple of num_kv_heads (GQA group size G)
+ *   num_kv_heads  KV heads; the retrieval/streaming type is per (layer, KV head)
+ *   head_dim      64 or 128
+ *   sink          attention-sink tokens kept by streaming heads (>= 0)
+ *   recent        recent tokens kept by streaming heads (>= 1); includes the
+ *                 query's own token, so a streaming query at position p attends
+ *                 to { j <= p : j < sink or p - j < recent }
+ *   max_len       capacity of every retrieval cache in tokens
+ *   softmax_scale 0 selects 1/sqrt(head_dim) */
+typedef struct duo_layout {
+    int32_t num_layers;
+    int32_t batch;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t head_dim;
+    int32_t sink;
+    int32_t recent;
+    int32_t reserved0;
+    int64_t max_len;
+    float softmax_scale;
+    int32_t reserved1;
+} duo_layout;
+
+/* Opaque host object: the layout, the per-layer head maps and lengths, and
+ * pointers into the caller's device buffer. */
+typedef struct duo_cache duo_cache;
+
+/* duo_cache_alloc — set up the two cache kinds of DuoAttention (a full cache per
+ * retrieval head, a constant-length sink + recent cache per streaming head;
+ * DuoAttention abstract) inside one caller-owned device buffer.
+ *   layout        shape (see duo_layout); copied
+ *   is_retrieval  host array [num_layers][num_kv_heads]: 1 = retrieval, 0 = streaming
+ *   dev_buf       device buffer of at least *required_bytes bytes, 256-byte
+ *                 aligned; NULL to only compute *required_bytes
+ *   buf_bytes     size of dev_buf
+ *   required_bytes out: bytes the cache needs (always written when non-NULL)
+ *   stream        stream on which the buffer is zero-filled
+ *   out           out: the new cache object (when dev_buf != NULL)
+ * Device layout inside dev_buf (offsets in required_bytes order):
+ *   retrieval K, V pools  [n_retrieval_heads_all_layers][batch][max_len][head_dim]
+ *   streaming K, V pools  [n_streaming_heads_all_layers][batch][sink+recent][head_dim]
+ *   streaming slot rule   position p < sink -> slot p; otherwise slot
+ *                         sink + (p - sink) mod recent (fixed sinks + a ring)
+ *   decode scratch        split-KV partial results, counters, an error word
+ * The caller keeps ownership of dev_buf and frees it after duo_cache_free. */
+DUO_API duo_status duo_cache_alloc(const duo_layout* layout, const uint8_t* is_retrieval, void* dev_buf,
+                           size_t buf_bytes, size_t* required_bytes, void* stream, duo_cache** out);
+
+/* duo_cache_free — release the host object (not the device buffer). NULL is allowed. */
+DUO_API duo_status duo_cache_free(duo_cache* cache);
+
+/* duo_cache_append — append n_tok tokens per sequence to every KV head of `layer`
+ * (the per-head cache update of DuoAttention: retrieval heads keep everything,
+ * streaming heads keep sinks and evict the oldest recent token).
+ *   k, v   device [batch][n_tok][num_kv_heads][head_dim] bf16, the tokens at
+ *          positions [len, len + n_tok) with len = duo_cache_len(layer)
+ *   n_tok  >= 0 (0 is a no-op)
+ * Retrieval heads write position p to slot p. Streaming heads write sink
+ * positions to their slots and only the last min(n_tok, recent) non-sink
+ * positions to their ring slots (earlier ones would be evicted within the call).
+ * DUO_ERR_CAPACITY if len + n_tok > max_len. Then len += n_tok. */
+DUO_API duo_status duo_cache_append(duo_cache* cache, int32_t layer, const void* k, const void* v, int64_t n_tok,
+                            void* stream);
+
+/* duo_prefill — attention of one prefill chunk of `layer` (DuoAttention
+ * pre-filling; chunked as in the chunked-prefill work the pages cite).
+ *   q      device [batch][n_tok][num_q_heads][head_dim], queries at positions
+ *          [len, len + n_tok) with len = duo_cache_len(layer)
+ *   k, v   device [batch][n_tok][num_kv_heads][head_dim], the chunk's own tokens
+ *   out    device [batch][n_tok][num_q_heads][head_dim], written
+ * Retrieval heads attend causally over the cache [0, len) and the chunk;
+ * streaming heads over the sinks and the recent window, read from the
+ * streaming cache for positions < len and from k/v for the chunk.
+ * Does NOT modify the cache: call duo_cache_append(layer, k, v, n_tok) after it.
+ * DUO_ERR_CAPACITY if a retrieval head could not hold len + n_tok tokens. */
+DUO_API duo_status duo_prefill(duo_cache* cache, int32_t layer, const void* q, const void* k, const void* v, void* out,
+                       int64_t n_tok, void* stream);
+
+/* duo_decode — one decoding step of `layer` (DuoAttention decoding).
+ *   q            device [batch][num_q_heads][head_dim], queries at position len
+ *   k_new, v_new device [batch][num_kv_heads][head_dim], the new token
+ *   out          device [batch][num_q_heads][head_dim], written
+ * Appends the new token to every head's cache (as duo_cache_append with one
+ * token), then attends: retrieval heads over positions [0, len], streaming
+ * heads over the sinks and the last `recent` positions. Then len += 1.
+ * Uses the cache's decode scratch: decode calls on one cache must not overlap
+ * on the device. DUO_ERR_CAPACITY if len + 1 > max_len. */
+DUO_API duo_status duo_decode(duo_cache* cache, int32_t layer, const void* q, const void* k_new, const void* v_new,
+                      void* out, void* stream);
+
+/* duo_cache_len — tokens appended so far to `layer` (host value; no sync). */
+DUO_API duo_status duo_cache_len(const duo_cache* cache, int32_t layer, int64_t* len);
+
+/* duo_cache_set_len — set the host-side length of `layer`, e.g. to restore a
+ * snapshot taken with duo_cache_len (the device contents are the caller's to
+ * restore). 0 <= len <= max_len. */
+DUO_API duo_status duo_cache_set_len(duo_cache* cache, int32_t layer, int64_t len);
+
+/* duo_cache_views — where one KV head's cache lives, for inspection.
+ *   k, v          out: device pointers to [batch][slots][head_dim] bf16
+ *   slots         out: max_len (retrieval) or sink + recent (streaming)
+ *   is_retrieval  out: 1 or 0
+ * Any out pointer may be NULL. */
+DUO_API duo_status duo_cache_views(const duo_cache* cache, int32_t layer, int32_t kv_head, void** k, void** v,
+                           int64_t* slots, int32_t* is_retrieval);
+
+/* duo_cache_error — read and clear the device-side error word of the cache
+ * (bit flags set by kernels whose bounded waits ran out). Synchronizes
+ * `stream`. *flags = 0 when no kernel reported an error. */
+DUO_API duo_status duo_cache_error(duo_cache* cache, void* stream, uint32_t* flags);
+
+/* duo_status_str — static description of a status code. */
+DUO_API const char* duo_status_str(duo_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DUO_H_ */

@@ -1,0 +1,99 @@
+// duo_internal.cuh — kernel parameter blocks and launch entry points shared by
+// the host ABI (duo_abi.cu) and the kernels (append.cu, decode.cu, prefill.cu).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/duo.h"
+
+namespace duo {
+
+using bf16 = __nv_bfloat16;
+
+// Per-layer KV-head map, passed by value: for every KV head its type and its
+// dense index in the retrieval pool or the streaming pool (over all layers).
+struct HeadMap {
+    int32_t pool_idx[DUO_MAX_KV_HEADS];
+    uint8_t is_retr[DUO_MAX_KV_HEADS];
+};
+
+// Where one layer's caches live.
+struct Pools {
+    bf16* rk;  // retrieval K pool [n_retr_all][B][max_len][D]
+    bf16* rv;
+    bf16* sk;  // streaming K pool [n_strm_all][B][W][D], W = sink + recent
+    bf16* sv;
+};
+
+// ------------------------------------------------------------------ append
+struct AppendParams {
+    const bf16* k;  // [B][n][Hkv][D]
+    const bf16* v;
+    Pools pools;
+    int64_t len;      // tokens cached before this call
+    int64_t n;        // tokens appended
+    int64_t max_len;
+    int32_t B, Hkv, D, S, R, W;
+    HeadMap heads;
+};
+cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
+
+// ------------------------------------------------------------------ decode
+constexpr int kDecodeMaxSplits = 256;
+constexpr int kDecodeThreads = 128;
+
+struct DecodeParams {
+    const bf16* q;      // [B][Hq][D]
+    const bf16* k_new;  // [B][Hkv][D]
+    const bf16* v_new;
+    bf16* out;          // [B][Hq][D]
+    Pools pools;
+    float* part_o;       // [B*Hkv*kDecodeMaxSplits][G][D]  normalised partial outputs
+    float* part_lse;     // [B*Hkv*kDecodeMaxSplits][G]     log2-sum-exp2 of the partial
+    uint32_t* counters;  // [B*Hkv] splits finished, reset by the merging CTA
+    uint32_t* err;
+    int64_t len;        // tokens cached before this step; the new token sits at position len
+    int64_t max_len;
+    int64_t split_rows;  // rows per retrieval split
+    int32_t nsplit;      // splits per retrieval (b, kv head)
+    int32_t B, Hq, Hkv, G, D, S, R, W;
+    int32_t n_retr, n_strm;  // retrieval / streaming KV heads in this layer
+    float scale_log2;        // softmax scale * log2(e)
+    int16_t retr_list[DUO_MAX_KV_HEADS];
+    int16_t strm_list[DUO_MAX_KV_HEADS];
+    HeadMap heads;
+};
+cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+
+// ------------------------------------------------------------------ prefill
+constexpr int kTileQ = 128;   // query rows per CTA (one TMEM lane each)
+constexpr int kTileK = 128;   // keys per KV tile
+
+struct PrefillParams {
+    bf16* out;  // [B][C][Hq][D]
+    uint32_t* err;
+    int64_t len;  // tokens cached before the chunk
+    int32_t C;    // chunk length
+    int32_t B, Hq, Hkv, G, D, S, R, W;
+    int32_t n_qt;      // ceil(C / kTileQ)
+    int32_t n_retr_q;  // retrieval query heads (listed first in qhead)
+    float scale_log2;
+    int16_t qhead[DUO_MAX_Q_HEADS];
+    HeadMap heads;
+};
+
+struct PrefillMaps {
+    CUtensorMap q;   // chunk q  (D, Hq, C, B), box (64, 1, 128, 1)
+    CUtensorMap k;   // chunk k  (D, Hkv, C, B)
+    CUtensorMap v;
+    CUtensorMap rk;  // retrieval pool (D, max_len, n_retr_all*B), box (64, 128, 1)
+    CUtensorMap rv;
+    CUtensorMap sk;  // streaming pool (D, W, n_strm_all*B), box (64, 128, 1)
+    CUtensorMap sv;
+};
+cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t s);
+
+}  // namespace duo
