@@ -141,6 +141,12 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self.proc = None
 
+    def samples(self) -> int:
+        try:
+            return sum(1 for line in open(self.path) if line.strip())
+        except OSError:
+            return 0
+
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
@@ -252,9 +258,17 @@ def run_gpu(args):
     step = Step(duo, w, device)
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
-    for _ in range(args.warmup):
-        step.run(sp)
-    torch.cuda.synchronize()
+    # Clocks are sampled from the start of warm-up to the end of the timed region
+    # (the timed region alone is shorter than nvidia-smi's start-up).
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_warm = time.perf_counter()
+    while True:
+        for _ in range(args.warmup):
+            step.run(sp)
+        torch.cuda.synchronize()
+        if clocks.samples() >= 3 or time.perf_counter() - t_warm > 10.0:
+            break
     if step.cache.error_flags() != 0:
         raise RuntimeError("device error flag set during warm-up")
 
@@ -262,8 +276,6 @@ def run_gpu(args):
     all_events = {kname: list(v) for kname, v in events.items()}
     for v in events.values():
         v.reverse()
-    clocks = ClockSampler(local)
-    clocks.start()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
     torch.cuda.synchronize()
@@ -325,7 +337,8 @@ def run_gpu(args):
                    "frac_of_measured_hbm": decode_gbs / peaks["hbm_gbs"], "frac_of_nominal_8000": decode_gbs / 8000.0},
         "append": {"gbs": append_gbs, "ms": t_ap},
         "roofline": roof, "kernels": kernels, "e2e": e2e,
-        "gpu_launches": step.launches_per_step * args.steps, "clocks": clk,
+        "gpu_launches": step.launches_per_step * args.steps,
+        "clocks": dict(clk, window="warm-up through timed region"),
     }
     if cpu is not None:
         res["cpu_baseline"] = cpu
