@@ -5,30 +5,10 @@
 #include <cstring>
 #include <mutex>
 #include <new>
-#include <vector>
 
 #include "duo_internal.cuh"
 
 using namespace duo;
-
-struct duo_cache {
-    duo_layout lay;
-    int32_t G = 1;
-    int32_t W = 0;
-    float scale = 0.f;
-    int device = 0;
-    int num_sms = 148;
-    std::vector<uint8_t> is_retr;       // [layers][Hkv]
-    std::vector<int32_t> pool_idx;      // [layers][Hkv] dense index within its pool
-    std::vector<int64_t> len;           // [layers]
-    int64_t n_retr_all = 0, n_strm_all = 0;
-    Pools pools{};
-    float* part_o = nullptr;
-    float* part_lse = nullptr;
-    uint32_t* counters = nullptr;
-    uint32_t* err = nullptr;
-    CUtensorMap map_rk{}, map_rv{}, map_sk{}, map_sv{};
-};
 
 namespace {
 
@@ -165,6 +145,7 @@ const char* duo_status_str(duo_status s) {
         case DUO_ERR_CUDA: return "CUDA call or kernel launch failed";
         case DUO_ERR_STATE: return "call not valid in the current state (device mismatch)";
         case DUO_ERR_DEVICE: return "a kernel reported a device-side error";
+        case DUO_ERR_SCRATCH_LIMIT: return "request exceeds the static decode scratch (DUO_STATIC_SCRATCH_BYTES)";
     }
     return "unknown status";
 }

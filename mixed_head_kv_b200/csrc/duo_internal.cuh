@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <vector>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -97,3 +98,23 @@ struct PrefillMaps {
 cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t s);
 
 }  // namespace duo
+
+// Host object behind the opaque duo_cache handle.
+struct duo_cache {
+    duo_layout lay;
+    int32_t G = 1;
+    int32_t W = 0;
+    float scale = 0.f;
+    int device = 0;
+    int num_sms = 148;
+    std::vector<uint8_t> is_retr;       // [layers][Hkv]
+    std::vector<int32_t> pool_idx;      // [layers][Hkv] dense index within its pool
+    std::vector<int64_t> len;           // [layers]
+    int64_t n_retr_all = 0, n_strm_all = 0;
+    duo::Pools pools{};
+    float* part_o = nullptr;
+    float* part_lse = nullptr;
+    uint32_t* counters = nullptr;
+    uint32_t* err = nullptr;
+    CUtensorMap map_rk{}, map_rv{}, map_sk{}, map_sv{};
+};
