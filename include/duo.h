@@ -53,7 +53,8 @@ typedef enum duo_status {
     DUO_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned */
     DUO_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed */
     DUO_ERR_STATE = 5,       /* call not valid in the cache's current state */
-    DUO_ERR_DEVICE = 6       /* a kernel reported a device-side error (see duo_cache_error) */
+    DUO_ERR_DEVICE = 6,      /* a kernel reported a device-side error (see duo_cache_error) */
+    DUO_ERR_SCRATCH_LIMIT = 7 /* the request needs more than DUO_STATIC_SCRATCH_BYTES */
 } duo_status;
 
 /* Largest head counts the kernels accept. */
@@ -173,6 +174,33 @@ DUO_API duo_status duo_cache_views(const duo_cache* cache, int32_t layer, int32_
  * (bit flags set by kernels whose bounded waits ran out). Synchronizes
  * `stream`. *flags = 0 when no kernel reported an error. */
 DUO_API duo_status duo_cache_error(duo_cache* cache, void* stream, uint32_t* flags);
+
+/* duo_decode_static_scratch — duo_decode for callers that cannot allocate device
+ * memory when they call in. The pages have no counterpart to this call: it is a
+ * deployment variant of the decode step.
+ *
+ * Some callers cannot call cudaMalloc at decode time: an inference-engine
+ * plugin that only gets a memory arena planned before the run, a serving loop
+ * that must not let cudaMalloc/cudaFree synchronize the device, or a process
+ * whose device-memory budget belongs to another allocator. This call computes
+ * exactly what duo_decode computes (same arguments, same cache update, same
+ * result within rounding), but keeps the split-KV partial results in one
+ * file-scope device array of DUO_STATIC_SCRATCH_BYTES instead of the cache's
+ * scratch region. It allocates nothing and calls no allocating routine.
+ *   - Every GPU that loads libduo holds the array until the process exits.
+ *   - All calls on a device share the array; it keeps the previous call's
+ *     contents (the call clears what must start at zero on `stream`). Calls
+ *     whose kernels overlap on the GPU race on it: issue them on one stream.
+ *   - The first call on a device looks up the array's address
+ *     (cudaGetSymbolAddress, device current): make it before any stream capture.
+ *   - DUO_ERR_SCRATCH_LIMIT when even one split per (sequence, retrieval head)
+ *     does not fit: batch * retrieval KV heads * G * (head_dim + 1) * 4 bytes
+ *     plus batch * num_kv_heads * 4 bytes of counters must stay below the limit.
+ *     Long contexts are served with fewer, longer splits when the full split
+ *     plan does not fit. */
+#define DUO_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
+DUO_API duo_status duo_decode_static_scratch(duo_cache* cache, int32_t layer, const void* q, const void* k_new,
+                                             const void* v_new, void* out, void* stream);
 
 /* duo_status_str — static description of a status code. */
 DUO_API const char* duo_status_str(duo_status status);

@@ -32,11 +32,14 @@ DUO_ERR_ALIGNMENT = 3
 DUO_ERR_CUDA = 4
 DUO_ERR_STATE = 5
 DUO_ERR_DEVICE = 6
+DUO_ERR_SCRATCH_LIMIT = 7
+DUO_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 DUO_MAX_Q_HEADS = 256
 DUO_MAX_KV_HEADS = 128
 
 EXPORTED = ("duo_cache_alloc", "duo_cache_free", "duo_cache_append", "duo_prefill", "duo_decode",
-            "duo_cache_len", "duo_cache_set_len", "duo_cache_views", "duo_cache_error", "duo_status_str")
+            "duo_cache_len", "duo_cache_set_len", "duo_cache_views", "duo_cache_error", "duo_status_str",
+            "duo_decode_static_scratch")
 
 
 class duo_layout(ctypes.Structure):
@@ -64,6 +67,8 @@ _lib.duo_prefill.restype = _ST
 _lib.duo_prefill.argtypes = [_P, _I32, _P, _P, _P, _P, _I64, _P]
 _lib.duo_decode.restype = _ST
 _lib.duo_decode.argtypes = [_P, _I32, _P, _P, _P, _P, _P]
+_lib.duo_decode_static_scratch.restype = _ST
+_lib.duo_decode_static_scratch.argtypes = [_P, _I32, _P, _P, _P, _P, _P]
 _lib.duo_cache_len.restype = _ST
 _lib.duo_cache_len.argtypes = [_P, _I32, ctypes.POINTER(_I64)]
 _lib.duo_cache_set_len.restype = _ST
@@ -143,6 +148,13 @@ def duo_prefill(handle, layer, q, k, v, out, n_tok, stream=None) -> int:
 
 def duo_decode(handle, layer, q, k_new, v_new, out, stream=None) -> int:
     return _lib.duo_decode(handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out), _stream(stream))
+
+
+def duo_decode_static_scratch(handle, layer, q, k_new, v_new, out, stream=None) -> int:
+    """duo_decode with its split-KV scratch in the library's static device array
+    (for callers that cannot allocate device memory at call time)."""
+    return _lib.duo_decode_static_scratch(handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+                                          _stream(stream))
 
 
 def duo_cache_len(handle, layer):

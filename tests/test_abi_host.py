@@ -121,6 +121,6 @@ def test_null_cache_rejected():
 
 
 def test_status_strings():
-    for s in range(7):
+    for s in range(8):
         assert duo.duo_status_str(s) and duo.duo_status_str(s) != "unknown status"
     assert duo.duo_status_str(99) == "unknown status"
