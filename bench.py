@@ -220,15 +220,15 @@ class Step:
                 e3.record()
             if st:
                 raise RuntimeError(f"prefill/append failed: {self.duo.duo_status_str(st)}")
+        if events is not None:
+            e0, e1 = events["decode"].pop()
+            e0.record()  # one pair around the decode loop: consecutive decodes overlap (PDL)
         for (p, qd, kd, vd, od) in self.dec:
-            if events is not None:
-                e0, e1 = events["decode"].pop()
-                e0.record()
             st = lib.duo_decode(self.h, 0, qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), stream_ptr)
-            if events is not None:
-                e1.record()
             if st:
                 raise RuntimeError(f"decode failed: {self.duo.duo_status_str(st)}")
+        if events is not None:
+            e1.record()
 
     def work(self):
         w, m = self.w, self.mask
@@ -242,7 +242,7 @@ def make_events(step, k):
     mk = lambda: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     return {"prefill": [mk() for _ in range(step.n_chunks * k)],
             "append": [mk() for _ in range(step.n_chunks * k)],
-            "decode": [mk() for _ in range(step.w.decode_steps * k)]}
+            "decode": [mk() for _ in range(k)]}
 
 
 def run_gpu(args):

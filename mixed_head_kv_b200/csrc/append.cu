@@ -14,6 +14,8 @@
 namespace duo {
 
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
+    grid_dependency_wait();  // launched with programmatic stream serialization
+    grid_launch_dependents();
     const int vec_per_row = p.D / 8;
     const int64_t total = static_cast<int64_t>(p.B) * p.n * p.Hkv * vec_per_row;
     const int64_t first_kept = p.len + p.n - p.R;  // ring positions below this are overwritten in-call
@@ -65,8 +67,7 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
     int64_t blocks = (total + threads - 1) / threads;
     const int64_t cap = static_cast<int64_t>(sms) * 8;  // grid-stride beyond 8 resident CTAs per SM
     if (blocks > cap) blocks = cap;
-    append_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(append_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, s, p);
 }
 
 }  // namespace duo

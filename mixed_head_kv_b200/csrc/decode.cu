@@ -11,11 +11,14 @@
 // so no CTA depends on another's cache write. Its ring slot held position
 // len - recent, which is outside the new query's window.
 //
-// Inside a CTA, 4 warps split the key range. A K/V row of D bf16 is read by
-// D/8 lanes with 16-byte non-caching loads (2 rows per warp instruction at
-// D = 128); each row is read once for all G query heads of its group. Scores
-// are reduced with warp shuffles; online softmax (exp2 domain) runs per lane
-// group and the groups/warps are merged at the end.
+// Memory path: each of the 4 warps streams a contiguous part of the item's
+// rows through its own 3-stage ring in shared memory, filled by bulk async
+// copies (cp.async.bulk, one K block and one V block of 4 KB per stage,
+// completion on an mbarrier). Each K/V row is read from HBM exactly once and
+// serves all G query heads of its group. A row of D bf16 is consumed by D/8
+// lanes (16 bytes each, conflict-free); scores are reduced with warp shuffles;
+// online softmax runs in the exp2 domain per lane group, and the groups, the
+// warps and finally the splits are merged with log-sum-exp weights.
 #include <cfloat>
 
 #include "duo_internal.cuh"
@@ -25,18 +28,32 @@ namespace duo {
 
 namespace {
 
-constexpr int kUnroll = 4;  // row groups in flight per warp iteration
 constexpr int kWarps = kDecodeThreads / 32;
+constexpr int kStages = 3;
+constexpr int kGroupRows = 4;  // row groups accumulated per register batch
 
-template <int D, int G>
+template <int D>
+struct Geom {
+    static constexpr int LPR = D / 8;                 // lanes per row
+    static constexpr int RPW = 32 / LPR;              // rows per warp instruction
+    static constexpr int BLK = 4096 / (D * 2);        // rows per 4 KB block
+    static constexpr int kBlockBytes = BLK * D * 2;   // one K (or V) block
+    static constexpr int kStageBytes = 2 * kBlockBytes;
+    static constexpr int kWarpBytes = kStages * kStageBytes;
+    static constexpr int kRingBytes = kWarps * kWarpBytes;  // 96 KB
+    static constexpr int kBarOff = kRingBytes;
+    static constexpr int kSmem = kBarOff + kWarps * kStages * 8 + 16;
+};
+
+template <int G>
 struct DecState {
     float m[G];
     float l[G];
     float o[G][8];
 };
 
-template <int D, int G>
-__device__ __forceinline__ void init_state(DecState<D, G>& st) {
+template <int G>
+__device__ __forceinline__ void init_state(DecState<G>& st) {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         st.m[h] = -INFINITY;
@@ -46,100 +63,79 @@ __device__ __forceinline__ void init_state(DecState<D, G>& st) {
     }
 }
 
-// Accumulate rows [r0, r1) (except `skip`) of one head's K/V into the state.
-// kbase/vbase point at row 0; row r lives at base + r * D.
-template <int D, int G>
-__device__ __forceinline__ void process_rows(DecState<D, G>& st, const float (&qf)[G][8], const bf16* kbase,
-                                             const bf16* vbase, int64_t r0, int64_t r1, int64_t skip) {
-    constexpr int LPR = D / 8;    // lanes per row
-    constexpr int RPW = 32 / LPR; // rows per warp instruction
-    const int lane = threadIdx.x & 31;
-    const int sub = lane % LPR;
-    const int rsub = lane / LPR;
-    for (int64_t base = r0; base < r1; base += kUnroll * RPW) {
-        uint4 kx[kUnroll], vx[kUnroll];
-        bool valid[kUnroll];
+// Fold U row groups (this lane's 16-byte slices of K and V rows) into the state.
+template <int D, int G, int U>
+__device__ __forceinline__ void accumulate(DecState<G>& st, const float (&qf)[G][8], const uint4 (&kx)[U],
+                                           const uint4 (&vx)[U], const bool (&valid)[U]) {
+    constexpr int LPR = D / 8;
+    float s[U][G];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t row = base + u * RPW + rsub;
-            valid[u] = (row < r1) && (row != skip);
-            if (valid[u]) {
-                kx[u] = ld_nc_v4(kbase + row * D + sub * 8);
-                vx[u] = ld_nc_v4(vbase + row * D + sub * 8);
-            } else {
-                kx[u] = make_uint4(0, 0, 0, 0);
-                vx[u] = make_uint4(0, 0, 0, 0);
-            }
-        }
-        float s[kUnroll][G];
+    for (int u = 0; u < U; ++u) {
+        const uint32_t w[4] = {kx[u].x, kx[u].y, kx[u].z, kx[u].w};
+        float kf[8];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t w[4] = {kx[u].x, kx[u].y, kx[u].z, kx[u].w};
-            float kf[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                kf[2 * i] = bf16lo_to_f32(w[i]);
-                kf[2 * i + 1] = bf16hi_to_f32(w[i]);
-            }
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                float acc = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc = fmaf(qf[h][e], kf[e], acc);
-                s[u][h] = acc;
-            }
-        }
-#pragma unroll
-        for (int off = LPR / 2; off >= 1; off >>= 1) {
-#pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) s[u][h] += __shfl_xor_sync(0xffffffffu, s[u][h], off);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            if (!valid[u]) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) s[u][h] = -INFINITY;
-            }
-        }
-        float vf[kUnroll][8];
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const uint32_t w[4] = {vx[u].x, vx[u].y, vx[u].z, vx[u].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                vf[u][2 * i] = bf16lo_to_f32(w[i]);
-                vf[u][2 * i + 1] = bf16hi_to_f32(w[i]);
-            }
+        for (int i = 0; i < 4; ++i) {
+            kf[2 * i] = bf16lo_to_f32(w[i]);
+            kf[2 * i + 1] = bf16hi_to_f32(w[i]);
         }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            float mb = s[0][h];
+            float acc = 0.f;
 #pragma unroll
-            for (int u = 1; u < kUnroll; ++u) mb = fmaxf(mb, s[u][h]);
-            const float mn = fmaxf(st.m[h], mb);
-            if (mn == -INFINITY) continue;  // nothing valid for this lane group yet
-            const float f = fast_exp2(st.m[h] - mn);  // 0 when the old max is -inf
-            st.m[h] = mn;
-            st.l[h] *= f;
+            for (int e = 0; e < 8; ++e) acc = fmaf(qf[h][e], kf[e], acc);
+            s[u][h] = acc;
+        }
+    }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) st.o[h][e] *= f;
+    for (int off = LPR / 2; off >= 1; off >>= 1) {
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const float pu = fast_exp2(s[u][h] - mn);
-                st.l[h] += pu;
+        for (int u = 0; u < U; ++u) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) st.o[h][e] = fmaf(pu, vf[u][e], st.o[h][e]);
-            }
+            for (int h = 0; h < G; ++h) s[u][h] += __shfl_xor_sync(0xffffffffu, s[u][h], off);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        if (!valid[u]) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) s[u][h] = -INFINITY;
+        }
+    }
+    float vf[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const uint32_t w[4] = {vx[u].x, vx[u].y, vx[u].z, vx[u].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            vf[u][2 * i] = bf16lo_to_f32(w[i]);
+            vf[u][2 * i + 1] = bf16hi_to_f32(w[i]);
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        float mb = s[0][h];
+#pragma unroll
+        for (int u = 1; u < U; ++u) mb = fmaxf(mb, s[u][h]);
+        const float mn = fmaxf(st.m[h], mb);
+        if (mn == -INFINITY) continue;  // nothing valid for this lane group yet
+        const float f = fast_exp2(st.m[h] - mn);  // 0 when the old max is -inf
+        st.m[h] = mn;
+        st.l[h] *= f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) st.o[h][e] *= f;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const float pu = fast_exp2(s[u][h] - mn);
+            st.l[h] += pu;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) st.o[h][e] = fmaf(pu, vf[u][e], st.o[h][e]);
         }
     }
 }
 
 // Merge the partial softmax state of the partner lane (xor `off`) into st.
-template <int D, int G>
-__device__ __forceinline__ void merge_lanes(DecState<D, G>& st, int off) {
+template <int G>
+__device__ __forceinline__ void merge_lanes(DecState<G>& st, int off) {
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         const float m2 = __shfl_xor_sync(0xffffffffu, st.m[h], off);
@@ -158,19 +154,94 @@ __device__ __forceinline__ void merge_lanes(DecState<D, G>& st, int off) {
     }
 }
 
+// Stream rows [r0, r1) (except `skip`) of one head through this warp's ring.
+// Returns false if a copy did not complete within the wait limit.
+template <int D, int G>
+__device__ bool warp_stream(DecState<G>& st, const float (&qf)[G][8], const bf16* kbase, const bf16* vbase,
+                            int64_t r0, int64_t r1, int64_t skip, uint32_t ring, uint32_t bars) {
+    using Gm = Geom<D>;
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % Gm::LPR;
+    const int rsub = lane / Gm::LPR;
+    const int64_t nblk = (r1 - r0 + Gm::BLK - 1) / Gm::BLK;
+    auto issue = [&](int64_t i) {
+        const int stg = static_cast<int>(i % kStages);
+        const int64_t a = r0 + i * Gm::BLK;
+        const int64_t n = (r1 - a < Gm::BLK) ? (r1 - a) : Gm::BLK;
+        const uint32_t bytes = static_cast<uint32_t>(n * D * 2);
+        const uint32_t bar = bars + 8u * stg;
+        const uint32_t dst = ring + stg * Gm::kStageBytes;
+        mbar_arrive_expect_tx(bar, 2 * bytes);
+        bulk_load(dst, kbase + a * D, bytes, bar);
+        bulk_load(dst + Gm::kBlockBytes, vbase + a * D, bytes, bar);
+    };
+    if (lane == 0) {
+        for (int64_t i = 0; i < nblk && i < kStages; ++i) issue(i);
+    }
+    for (int64_t i = 0; i < nblk; ++i) {
+        const int stg = static_cast<int>(i % kStages);
+        if (!mbar_wait(bars + 8u * stg, static_cast<uint32_t>((i / kStages) & 1), nullptr)) {
+            // Give the copies still in flight one more bounded wait before the
+            // CTA moves on (and later reuses this shared memory).
+            for (int64_t j = i + 1; j < nblk && j < i + kStages; ++j)
+                mbar_wait(bars + 8u * static_cast<uint32_t>(j % kStages), static_cast<uint32_t>((j / kStages) & 1),
+                          nullptr);
+            return false;
+        }
+        const int64_t a = r0 + i * Gm::BLK;
+        const int rows = static_cast<int>((r1 - a < Gm::BLK) ? (r1 - a) : Gm::BLK);
+        const uint32_t kst = ring + stg * Gm::kStageBytes;
+        const uint32_t vst = kst + Gm::kBlockBytes;
+#pragma unroll
+        for (int u0 = 0; u0 < Gm::BLK / Gm::RPW; u0 += kGroupRows) {
+            uint4 kx[kGroupRows], vx[kGroupRows];
+            bool valid[kGroupRows];
+#pragma unroll
+            for (int u = 0; u < kGroupRows; ++u) {
+                const int row = (u0 + u) * Gm::RPW + rsub;
+                valid[u] = row < rows && (a + row) != skip;
+                const uint32_t off = static_cast<uint32_t>(row * D * 2 + sub * 16);
+                kx[u] = valid[u] ? lds128(kst + off) : make_uint4(0, 0, 0, 0);
+                vx[u] = valid[u] ? lds128(vst + off) : make_uint4(0, 0, 0, 0);
+            }
+            accumulate<D, G, kGroupRows>(st, qf, kx, vx, valid);
+        }
+        __syncwarp();
+        if (lane == 0 && i + kStages < nblk) {
+            fence_proxy_async_smem();  // our generic reads of this stage precede the async refill
+            issue(i + kStages);
+        }
+    }
+    return true;
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams p) {
-    constexpr int LPR = D / 8;
-    __shared__ float sm_m[kWarps][G];
-    __shared__ float sm_l[kWarps][G];
-    __shared__ float sm_o[kWarps][G][D];
-    __shared__ float sm_w[G][kDecodeMaxSplits];
-    __shared__ int sm_last;
+    using Gm = Geom<D>;
+    constexpr int LPR = Gm::LPR;
+    extern __shared__ __align__(128) uint8_t smem[];
+    // After the streaming phase the ring is reused for the cross-warp merge.
+    float* sm_m = reinterpret_cast<float*>(smem);                 // [kWarps][G]
+    float* sm_l = sm_m + kWarps * G;                              // [kWarps][G]
+    float* sm_o = sm_l + kWarps * G;                              // [kWarps][G][D]
+    float* sm_w = sm_o + kWarps * G * D;                          // [G][kDecodeMaxSplits]
+    int* sm_last = reinterpret_cast<int*>(smem + Gm::kBarOff + kWarps * kStages * 8);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int sub = lane % LPR;
+    const uint32_t ring = smem_u32(smem) + warp * Gm::kWarpBytes;
+    const uint32_t bars = smem_u32(smem) + Gm::kBarOff + warp * kStages * 8;
+    if (lane == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(bars + 8u * s, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    // Launched with programmatic stream serialization: everything above overlaps
+    // the previous kernel's tail; no global memory is touched before this wait.
+    grid_dependency_wait();
+    grid_launch_dependents();
 
     const int n_retr_items = p.B * p.n_retr * p.nsplit;
     const bool is_retr = static_cast<int>(blockIdx.x) < n_retr_items;
@@ -242,27 +313,35 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
         }
     }
 
-    DecState<D, G> st;
+    DecState<G> st;
     init_state(st);
     const int64_t n_rows = r1 - r0;
-    const int64_t per_warp = (n_rows + kWarps - 1) / kWarps;
+    const int64_t per_warp = ((n_rows + kWarps - 1) / kWarps + Gm::BLK - 1) / Gm::BLK * Gm::BLK;
     const int64_t w0 = r0 + warp * per_warp;
     const int64_t w1 = (w0 + per_warp < r1) ? (w0 + per_warp) : r1;
-    if (w0 < w1) process_rows<D, G>(st, qf, kbase, vbase, w0, w1, skip);
-    if (owns_new && warp == 0) process_rows<D, G>(st, qf, knew, vnew, 0, 1, -1);
+    bool ok = true;
+    if (w0 < w1) ok = warp_stream<D, G>(st, qf, kbase, vbase, w0, w1, skip, ring, bars);
+    if (!ok && lane == 0) atomicOr(p.err, kErrDecodeCopy);
+    if (owns_new && warp == 0) {
+        uint4 kx[1] = {ld_nc_v4(knew + sub * 8)};
+        uint4 vx[1] = {ld_nc_v4(vnew + sub * 8)};
+        bool valid[1] = {lane < LPR};
+        accumulate<D, G, 1>(st, qf, kx, vx, valid);
+    }
 
     // Merge the row groups of the warp, then the warps.
 #pragma unroll
-    for (int off = LPR; off < 32; off <<= 1) merge_lanes<D, G>(st, off);
+    for (int off = LPR; off < 32; off <<= 1) merge_lanes<G>(st, off);
+    __syncthreads();  // every warp is done with its ring: reuse it for the merge
     if (lane < LPR) {
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             if (lane == 0) {
-                sm_m[warp][h] = st.m[h];
-                sm_l[warp][h] = st.l[h];
+                sm_m[warp * G + h] = st.m[h];
+                sm_l[warp * G + h] = st.l[h];
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) sm_o[warp][h][sub * 8 + e] = st.o[h][e];
+            for (int e = 0; e < 8; ++e) sm_o[(warp * G + h) * D + sub * 8 + e] = st.o[h][e];
         }
     }
     __syncthreads();
@@ -274,13 +353,13 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
         const int d = idx % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w][h]);
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w * G + h]);
         float Lsum = 0.f, O = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            const float f = fast_exp2(sm_m[w][h] - M);
-            Lsum += f * sm_l[w][h];
-            O += f * sm_o[w][h][d];
+            const float f = fast_exp2(sm_m[w * G + h] - M);
+            Lsum += f * sm_l[w * G + h];
+            O += f * sm_o[(w * G + h) * D + d];
         }
         if (final_now) {
             p.out[(static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d] = __float2bfloat16_rn(O / Lsum);
@@ -296,49 +375,94 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     __syncthreads();
     if (tid == 0) {
         const uint32_t prev = atomicAdd(&p.counters[b * p.Hkv + g], 1u);
-        sm_last = (prev == static_cast<uint32_t>(p.nsplit - 1));
+        *sm_last = (prev == static_cast<uint32_t>(p.nsplit - 1));
     }
     __syncthreads();
-    if (!sm_last) return;
+    if (!*sm_last) return;
     __threadfence();
+    // The partials of this (b, KV head) are contiguous: [nsplit][G][D] floats and
+    // [nsplit][G] log-sum-exps. Weights first, then a coalesced float4 pass in
+    // which each thread folds an independent subset of the splits.
     const int64_t item0 = (static_cast<int64_t>(b) * p.n_retr + ri) * p.nsplit;
+    const int ns = p.nsplit;
     for (int h = warp; h < G; h += kWarps) {
         float M = -INFINITY;
-        for (int s = lane; s < p.nsplit; s += 32) M = fmaxf(M, __ldcg(p.part_lse + (item0 + s) * G + h));
+        for (int s = lane; s < ns; s += 32) {
+            const float x = __ldcg(p.part_lse + (item0 + s) * G + h);
+            sm_w[h * kDecodeMaxSplits + s] = x;
+            M = fmaxf(M, x);
+        }
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
         float sum = 0.f;
-        for (int s = lane; s < p.nsplit; s += 32) {
-            const float w = fast_exp2(__ldcg(p.part_lse + (item0 + s) * G + h) - M);
-            sm_w[h][s] = w;
+        for (int s = lane; s < ns; s += 32) {
+            const float w = fast_exp2(sm_w[h * kDecodeMaxSplits + s] - M);
+            sm_w[h * kDecodeMaxSplits + s] = w;
             sum += w;
         }
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
         const float inv = 1.f / sum;
-        for (int s = lane; s < p.nsplit; s += 32) sm_w[h][s] *= inv;
+        for (int s = lane; s < ns; s += 32) sm_w[h * kDecodeMaxSplits + s] *= inv;
     }
     __syncthreads();
-    for (int idx = tid; idx < G * D; idx += kDecodeThreads) {
-        const int h = idx / D;
-        const int d = idx % D;
-        float acc = 0.f;
-        for (int s = 0; s < p.nsplit; ++s) acc = fmaf(sm_w[h][s], __ldcg(p.part_o + ((item0 + s) * G + h) * D + d), acc);
-        p.out[(static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d] = __float2bfloat16_rn(acc);
+    constexpr int kUnits = G * D / 4;  // float4 units of one split's partial
+    constexpr int kRep = kUnits >= kDecodeThreads ? 1 : kDecodeThreads / kUnits;
+    float* sm_red = sm_w + G * kDecodeMaxSplits;  // [kRep][kUnits] float4
+    const float4* po = reinterpret_cast<const float4*>(p.part_o + item0 * G * D);
+    for (int u = tid % kUnits; u < kUnits; u += kDecodeThreads) {
+        const int h = (u * 4) / D;
+        const int rep = tid / kUnits;  // < kRep
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int s = rep; s < ns; s += kRep) {
+            const float w = sm_w[h * kDecodeMaxSplits + s];
+            const float4 x = __ldcg(po + static_cast<int64_t>(s) * kUnits + u);
+            acc.x = fmaf(w, x.x, acc.x);
+            acc.y = fmaf(w, x.y, acc.y);
+            acc.z = fmaf(w, x.z, acc.z);
+            acc.w = fmaf(w, x.w, acc.w);
+        }
+        reinterpret_cast<float4*>(sm_red)[rep * kUnits + u] = acc;
+    }
+    __syncthreads();
+    for (int u = tid; u < kUnits; u += kDecodeThreads) {
+        float4 acc = reinterpret_cast<const float4*>(sm_red)[u];
+        for (int r = 1; r < kRep; ++r) {
+            const float4 x = reinterpret_cast<const float4*>(sm_red)[r * kUnits + u];
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+        }
+        const int h = (u * 4) / D;
+        const int d = (u * 4) % D;
+        bf16* o = p.out + (static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d;
+        *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
     }
     if (tid == 0) p.counters[b * p.Hkv + g] = 0u;  // ready for the next step (stream-ordered)
+}
+
+template <int D, int G>
+cudaError_t launch_dg(const DecodeParams& p, unsigned grid, cudaStream_t s) {
+    constexpr int smem = Geom<D>::kSmem;
+    static_assert((kWarps * 2 * G + kWarps * G * D + G * kDecodeMaxSplits) * 4 + 16 * 2 * kDecodeThreads +
+                          16 * G * D / 4 <= Geom<D>::kRingBytes,
+                  "merge arrays must fit in the ring");
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(decode_kernel<D, G>, dim3(grid), dim3(kDecodeThreads), smem, s, p);
 }
 
 template <int D>
 cudaError_t launch_d(const DecodeParams& p, unsigned grid, cudaStream_t s) {
     switch (p.G) {
-        case 1: decode_kernel<D, 1><<<grid, kDecodeThreads, 0, s>>>(p); break;
-        case 2: decode_kernel<D, 2><<<grid, kDecodeThreads, 0, s>>>(p); break;
-        case 4: decode_kernel<D, 4><<<grid, kDecodeThreads, 0, s>>>(p); break;
-        case 8: decode_kernel<D, 8><<<grid, kDecodeThreads, 0, s>>>(p); break;
+        case 1: return launch_dg<D, 1>(p, grid, s);
+        case 2: return launch_dg<D, 2>(p, grid, s);
+        case 4: return launch_dg<D, 4>(p, grid, s);
+        case 8: return launch_dg<D, 8>(p, grid, s);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace

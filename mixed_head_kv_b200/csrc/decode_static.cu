@@ -99,16 +99,10 @@ extern "C" duo_status duo_decode_static_scratch(duo_cache* c, int32_t layer, con
 
     // Same split plan as duo_decode, then limited to what the array holds.
     const int64_t rows = p.len + 1;
-    int64_t nsplit = 1;
+    int64_t nsplit = plan_decode_splits(L.batch, p.n_retr, p.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms);
     const size_t counters_bytes = round256(static_cast<size_t>(L.batch) * L.num_kv_heads * sizeof(uint32_t));
     if (p.n_retr > 0) {
         const int64_t pairs = static_cast<int64_t>(L.batch) * p.n_retr;
-        const int64_t target = static_cast<int64_t>(c->num_sms) * 4;
-        nsplit = (target + pairs - 1) / pairs;
-        const int64_t by_rows = (rows + 255) / 256;
-        if (nsplit > by_rows) nsplit = by_rows;
-        if (nsplit > kDecodeMaxSplits) nsplit = kDecodeMaxSplits;
-        if (nsplit < 1) nsplit = 1;
         // Bytes per split: partial outputs and their log-sum-exp, for every (b, retrieval head, query head).
         const size_t per_split = static_cast<size_t>(pairs) * p.G * (static_cast<size_t>(p.D) + 1) * sizeof(float);
         const size_t room = kStaticBytes - counters_bytes - 256;  // 256: alignment of the second region

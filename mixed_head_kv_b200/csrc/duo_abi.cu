@@ -370,18 +370,8 @@ duo_status duo_decode(duo_cache* c, int32_t layer, const void* q, const void* k_
         if (p.heads.is_retr[g]) p.retr_list[p.n_retr++] = static_cast<int16_t>(g);
         else p.strm_list[p.n_strm++] = static_cast<int16_t>(g);
     }
-    // Split plan: about 4 CTAs per SM over the retrieval rows, at least 256 rows per split.
     const int64_t rows = p.len + 1;
-    int64_t nsplit = 1;
-    if (p.n_retr > 0) {
-        const int64_t pairs = static_cast<int64_t>(L.batch) * p.n_retr;
-        const int64_t target = static_cast<int64_t>(c->num_sms) * 4;
-        nsplit = (target + pairs - 1) / pairs;
-        const int64_t by_rows = (rows + 255) / 256;
-        if (nsplit > by_rows) nsplit = by_rows;
-        if (nsplit > kDecodeMaxSplits) nsplit = kDecodeMaxSplits;
-        if (nsplit < 1) nsplit = 1;
-    }
+    const int64_t nsplit = plan_decode_splits(L.batch, p.n_retr, p.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms);
     p.split_rows = (rows + nsplit - 1) / nsplit;
     p.nsplit = static_cast<int32_t>((rows + p.split_rows - 1) / p.split_rows);
     if (launch_decode(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUO_ERR_CUDA;

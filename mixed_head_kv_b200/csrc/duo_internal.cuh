@@ -14,6 +14,24 @@ namespace duo {
 
 using bf16 = __nv_bfloat16;
 
+// Launch `kernel` on stream `s` with programmatic stream serialization: its
+// CTAs may start while the previous kernel of the stream drains; the kernel
+// itself waits (griddepcontrol.wait) before touching dependent memory.
+template <typename Kernel, typename Params>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, const Params& p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 // Per-layer KV-head map, passed by value: for every KV head its type and its
 // dense index in the retrieval pool or the streaming pool (over all layers).
 struct HeadMap {
@@ -45,6 +63,39 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 // ------------------------------------------------------------------ decode
 constexpr int kDecodeMaxSplits = 256;
 constexpr int kDecodeThreads = 128;
+
+constexpr int kDecodeCtasPerSm = 2;  // residency of decode_kernel (96 KB of shared memory each)
+
+// Splits per retrieval (b, KV head) for one decode step. Every CTA streams
+// its rows at about the same rate, so the step takes about
+//   waves * (rows of the longest CTA + a fixed per-CTA cost),
+// waves = ceil(CTAs / resident slots). The streaming items are one CTA of up to
+// sink + recent rows each. Pick the split count (>= 256 rows per split, at most
+// kDecodeMaxSplits) that minimises that estimate.
+inline int64_t plan_decode_splits(int64_t batch, int64_t n_retr, int64_t n_strm, int64_t rows, int64_t strm_rows,
+                                  int num_sms) {
+    if (n_retr <= 0) return 1;
+    constexpr int64_t kCtaCostRows = 64;
+    const int64_t pairs = batch * n_retr;
+    const int64_t strm_items = batch * n_strm;
+    const int64_t slots = static_cast<int64_t>(num_sms) * kDecodeCtasPerSm;
+    int64_t max_split = (rows + 255) / 256;
+    if (max_split > kDecodeMaxSplits) max_split = kDecodeMaxSplits;
+    if (max_split < 1) max_split = 1;
+    int64_t best = 1, best_cost = -1;
+    for (int64_t ns = 1; ns <= max_split; ++ns) {
+        const int64_t ctas = pairs * ns + strm_items;
+        const int64_t waves = (ctas + slots - 1) / slots;
+        int64_t longest = (rows + ns - 1) / ns;
+        if (strm_items > 0 && strm_rows > longest) longest = strm_rows;
+        const int64_t cost = waves * (longest + kCtaCostRows);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best = ns;
+        }
+    }
+    return best;
+}
 
 struct DecodeParams {
     const bf16* q;      // [B][Hq][D]

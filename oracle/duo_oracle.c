@@ -56,19 +56,20 @@ int duo_oracle_key_allowed(int is_retrieval, int64_t p, int64_t j, int64_t sink,
     return (j < sink) || (p - j < recent);
 }
 
-/* Attention of one query row over an explicit list of key rows.
- * q[D]; keys/vals: n rows of D bf16 each, row i at keys + i*D.
- * out[D] receives sum_i a_i v_i; *wsum receives sum_i a_i (1 up to rounding).
- * Returns 0, or -1 when the list is empty or allocation fails. */
-int duo_oracle_attend_rows(const uint16_t* q, const uint16_t* keys, const uint16_t* vals,
-                           int64_t n, int D, double scale, double* out, double* wsum) {
+/* Softmax attention of one query row over the key/value rows listed in idx:
+ * row idx[i] of keys/vals (D bf16 each). out[D] receives sum_i a_i v_i and
+ * *wsum receives sum_i a_i (1 up to rounding). Returns 0, or -1 when the list
+ * is empty or allocation fails. */
+static int attend_indexed(const uint16_t* q, const uint16_t* keys, const uint16_t* vals, const int64_t* idx,
+                          int64_t n, int D, double scale, double* out, double* wsum) {
     if (n <= 0) return -1;
     double* s = (double*)malloc(sizeof(double) * (size_t)n);
     if (!s) return -1;
     double m = -INFINITY;
     for (int64_t i = 0; i < n; ++i) {
+        const uint16_t* kr = keys + idx[i] * D;
         double dot = 0.0;
-        for (int d = 0; d < D; ++d) dot += bf16_to_double(q[d]) * bf16_to_double(keys[i * D + d]);
+        for (int d = 0; d < D; ++d) dot += bf16_to_double(q[d]) * bf16_to_double(kr[d]);
         s[i] = scale * dot;
         if (s[i] > m) m = s[i];
     }
@@ -80,13 +81,27 @@ int duo_oracle_attend_rows(const uint16_t* q, const uint16_t* keys, const uint16
     for (int d = 0; d < D; ++d) out[d] = 0.0;
     double total = 0.0;
     for (int64_t i = 0; i < n; ++i) {
+        const uint16_t* vr = vals + idx[i] * D;
         double a = s[i] / denom;
         total += a;
-        for (int d = 0; d < D; ++d) out[d] += a * bf16_to_double(vals[i * D + d]);
+        for (int d = 0; d < D; ++d) out[d] += a * bf16_to_double(vr[d]);
     }
     if (wsum) *wsum = total;
     free(s);
     return 0;
+}
+
+/* Attention of one query row over an explicit list of n key/value rows
+ * (row i at keys + i*D). */
+int duo_oracle_attend_rows(const uint16_t* q, const uint16_t* keys, const uint16_t* vals,
+                           int64_t n, int D, double scale, double* out, double* wsum) {
+    if (n <= 0) return -1;
+    int64_t* idx = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
+    if (!idx) return -1;
+    for (int64_t i = 0; i < n; ++i) idx[i] = i;
+    int rc = attend_indexed(q, keys, vals, idx, n, D, scale, out, wsum);
+    free(idx);
+    return rc;
 }
 
 /* Attention of one query at absolute position p of one head over the full
@@ -99,19 +114,13 @@ static int attend_masked(const uint16_t* q, const uint16_t* k_hist, const uint16
     int64_t n = 0;
     for (int64_t j = 0; j <= last; ++j) n += duo_oracle_key_allowed(is_retrieval, p, j, sink, recent);
     if (n == 0) return -1;
-    uint16_t* kk = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * D));
-    uint16_t* vv = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(n * D));
-    if (!kk || !vv) { free(kk); free(vv); return -1; }
+    int64_t* idx = (int64_t*)malloc(sizeof(int64_t) * (size_t)n);
+    if (!idx) return -1;
     int64_t c = 0;
-    for (int64_t j = 0; j <= last; ++j) {
-        if (!duo_oracle_key_allowed(is_retrieval, p, j, sink, recent)) continue;
-        memcpy(kk + c * D, k_hist + j * D, sizeof(uint16_t) * (size_t)D);
-        memcpy(vv + c * D, v_hist + j * D, sizeof(uint16_t) * (size_t)D);
-        ++c;
-    }
-    int rc = duo_oracle_attend_rows(q, kk, vv, n, D, scale, out, wsum);
-    free(kk);
-    free(vv);
+    for (int64_t j = 0; j <= last; ++j)
+        if (duo_oracle_key_allowed(is_retrieval, p, j, sink, recent)) idx[c++] = j;
+    int rc = attend_indexed(q, k_hist, v_hist, idx, n, D, scale, out, wsum);
+    free(idx);
     return rc;
 }
 
