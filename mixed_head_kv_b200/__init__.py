@@ -3,7 +3,7 @@
 Argument marshalling only: every step of the computation runs in the CUDA
 kernels of libduo.so. PyTorch supplies device memory and streams. The module
 refuses to load when libduo.so has not been built (run
-`python -m mixed_head_kv_b200.build` or `__graft_entry__.build()`); there is
+`python mixed_head_kv_b200/build.py` or `__graft_entry__.build()`); there is
 no fallback path.
 
 Functions keep the C names: duo_cache_alloc, duo_cache_free, duo_cache_append,
@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libduo.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libduo.so is not built at {LIB_PATH}; run `python -m mixed_head_kv_b200.build`")
+    raise ImportError(f"libduo.so is not built at {LIB_PATH}; run `python mixed_head_kv_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -205,7 +205,10 @@ class DuoCache:
             self.handle = None
 
     def __del__(self):
-        self.close()
+        try:
+            self.close()
+        except Exception:  # interpreter shutdown: module globals may already be gone
+            pass
 
     def append(self, layer, k, v, stream=None):
         _check(duo_cache_append(self.handle, layer, k, v, k.shape[1], stream), "duo_cache_append")
