@@ -360,28 +360,60 @@ def load_traffic(kernel: str):
 
 
 def run_e2e(duo, step, args, sp, device):
-    """The same step from pinned host buffers: H2D of every input, the ABI calls, D2H of every output."""
-    hc = [(qc.cpu().pin_memory(), kc.cpu().pin_memory(), vc.cpu().pin_memory(), torch.empty_like(oc, device="cpu").pin_memory())
-          for (_p, _n, qc, kc, vc, oc) in step.chunks]
-    hd = [(qd.cpu().pin_memory(), kd.cpu().pin_memory(), vd.cpu().pin_memory(), torch.empty_like(od, device="cpu").pin_memory())
-          for (_p, qd, kd, vd, od) in step.dec]
+    """The same step from pinned host buffers through the same C ABI: every input is
+    copied host -> device and every output device -> host inside the timed region.
+    Copies run on their own streams and overlap the kernels: the upload of chunk i+1
+    runs while chunk i computes, and each output is read back as soon as it is ready."""
+    lib = duo._lib
+    hc = [(qc.cpu().pin_memory(), kc.cpu().pin_memory(), vc.cpu().pin_memory(),
+           torch.empty_like(oc, device="cpu").pin_memory()) for (_p, _n, qc, kc, vc, oc) in step.chunks]
+    hd = [(qd.cpu().pin_memory(), kd.cpu().pin_memory(), vd.cpu().pin_memory(),
+           torch.empty_like(od, device="cpu").pin_memory()) for (_p, qd, kd, vd, od) in step.dec]
     h2d = sum(a.numel() * 2 + b.numel() * 2 + c.numel() * 2 for a, b, c, _ in hc + hd)
     d2h = sum(o.numel() * 2 for *_x, o in hc + hd)
+    main = torch.cuda.current_stream()
+    up = torch.cuda.Stream(device=device)
+    down = torch.cuda.Stream(device=device)
+    n_c = len(step.chunks)
+    ev_in = [torch.cuda.Event() for _ in range(n_c + 1)]
+    ev_out = [torch.cuda.Event() for _ in range(n_c + 1)]
 
     def one():
-        for (hq, hk, hv, ho), (_p, _n, qc, kc, vc, oc) in zip(hc, step.chunks):
-            qc.copy_(hq, non_blocking=True)
-            kc.copy_(hk, non_blocking=True)
-            vc.copy_(hv, non_blocking=True)
-        for (hq, hk, hv, ho), (_p, qd, kd, vd, od) in zip(hd, step.dec):
-            qd.copy_(hq, non_blocking=True)
-            kd.copy_(hk, non_blocking=True)
-            vd.copy_(hv, non_blocking=True)
-        step.run(sp)
-        for (hq, hk, hv, ho), (_p, _n, qc, kc, vc, oc) in zip(hc, step.chunks):
-            ho.copy_(oc, non_blocking=True)
-        for (hq, hk, hv, ho), (_p, qd, kd, vd, od) in zip(hd, step.dec):
-            ho.copy_(od, non_blocking=True)
+        duo.duo_cache_set_len(step.h, 0, 0)
+        with torch.cuda.stream(up):
+            for i, ((hq, hk, hv, _ho), (_p, _n, qc, kc, vc, _oc)) in enumerate(zip(hc, step.chunks)):
+                qc.copy_(hq, non_blocking=True)
+                kc.copy_(hk, non_blocking=True)
+                vc.copy_(hv, non_blocking=True)
+                ev_in[i].record(up)
+            for (hq, hk, hv, _ho), (_p, qd, kd, vd, _od) in zip(hd, step.dec):
+                qd.copy_(hq, non_blocking=True)
+                kd.copy_(hk, non_blocking=True)
+                vd.copy_(hv, non_blocking=True)
+            ev_in[n_c].record(up)
+        for i, (p0, n, qc, kc, vc, oc) in enumerate(step.chunks):
+            main.wait_event(ev_in[i])
+            st = lib.duo_prefill(step.h, 0, qc.data_ptr(), kc.data_ptr(), vc.data_ptr(), oc.data_ptr(), n, sp)
+            ev_out[i].record(main)
+            st |= lib.duo_cache_append(step.h, 0, kc.data_ptr(), vc.data_ptr(), n, sp)
+            if st:
+                raise RuntimeError(f"prefill/append failed: {duo.duo_status_str(st)}")
+        main.wait_event(ev_in[n_c])
+        for (p, qd, kd, vd, od) in step.dec:
+            st = lib.duo_decode(step.h, 0, qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), sp)
+            if st:
+                raise RuntimeError(f"decode failed: {duo.duo_status_str(st)}")
+        ev_out[n_c].record(main)
+        with torch.cuda.stream(down):
+            for i, ((_hq, _hk, _hv, ho), (_p, _n, _qc, _kc, _vc, oc)) in enumerate(zip(hc, step.chunks)):
+                down.wait_event(ev_out[i])
+                ho.copy_(oc, non_blocking=True)
+            down.wait_event(ev_out[n_c])
+            for (_hq, _hk, _hv, ho), (_p, _qd, _kd, _vd, od) in zip(hd, step.dec):
+                ho.copy_(od, non_blocking=True)
+        # the next step reuses the device inputs/outputs: order it after this step's copies
+        main.wait_stream(down)
+        up.wait_stream(main)
 
     for _ in range(max(1, args.warmup)):
         one()
@@ -389,15 +421,17 @@ def run_e2e(duo, step, args, sp, device):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(device)
     t0.record()
+    up.wait_stream(main)  # the first uploads start after t0
     for _ in range(args.steps):
         one()
-    t1.record()
+    t1.record()  # one() ends with the main stream waiting for the last read-back
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1), device) / args.steps
     world = dist_env()[0]
     tok = step.w.batch * step.T
     return {"value": world * tok / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "overlap": "uploads, kernels and read-backs on separate streams"}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) timing

@@ -86,7 +86,7 @@ __device__ __forceinline__ uint32_t tmem_o(int x) { return x ? 384u : 256u; }
 // What one work item attends to.
 struct Item {
     int b, head, g, tp, retr, pool;
-    int q0[2];    // first chunk row of tile A / B
+    int q0a, q0b;  // first chunk row of tile A / B (scalars: no local memory)
     int n_cache;  // cache tiles
     int src_cache;
     int a;        // streaming: chunk tiles holding chunk-resident sinks
@@ -115,8 +115,8 @@ __device__ __forceinline__ Item make_item(const PrefillParams& p) {
     it.g = it.head / p.G;
     it.retr = p.heads.is_retr[it.g];
     it.pool = p.heads.pool_idx[it.g];
-    it.q0[0] = it.tp * 2 * kTileQ;
-    it.q0[1] = it.q0[0] + kTileQ;
+    it.q0a = it.tp * 2 * kTileQ;
+    it.q0b = it.q0a + kTileQ;
     const int qt_last = (2 * it.tp + 1 < p.n_qt) ? 2 * it.tp + 1 : 2 * it.tp;
     const int64_t L = p.len;
     if (it.retr) {
@@ -129,7 +129,7 @@ __device__ __forceinline__ Item make_item(const PrefillParams& p) {
         it.src_cache = 1;
         int64_t slots = 0;
         if (L > 0) {
-            const bool band_in_cache = (L > p.S) && (it.q0[0] < p.R - 1);
+            const bool band_in_cache = (L > p.S) && (it.q0a < p.R - 1);
             slots = band_in_cache ? (L < p.W ? L : p.W) : (L < p.S ? L : p.S);
         }
         it.n_cache = static_cast<int>((slots + kTileK - 1) / kTileK);
@@ -139,7 +139,7 @@ __device__ __forceinline__ Item make_item(const PrefillParams& p) {
             a = static_cast<int>((sink_rows + kTileK - 1) / kTileK);
             if (a > qt_last + 1) a = qt_last + 1;
         }
-        const int band_lo = it.q0[0] - p.R + 1 > 0 ? it.q0[0] - p.R + 1 : 0;
+        const int band_lo = it.q0a - p.R + 1 > 0 ? it.q0a - p.R + 1 : 0;
         const int tb = band_lo / kTileK;
         it.a = a;
         it.b0 = a > tb ? a : tb;
@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(bar(kQFull), 2 * Lay::kTile);
             for (int x = 0; x < 2; ++x)
                 for (int kb = 0; kb < Lay::kColBlocks; ++kb)
-                    tma_load_4d(sQ(x) + kb * kTileBytesPerColBlock, &maps.q, bar(kQFull), kb * 64, it.head, it.q0[x],
+                    tma_load_4d(sQ(x) + kb * kTileBytesPerColBlock, &maps.q, bar(kQFull), kb * 64, it.head, x ? it.q0b : it.q0a,
                                 it.b);
             int issued = 0;
             for (int j = 0; j < n; ++j) {
@@ -417,7 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ softmax warps
         const int x = warp >> 2;          // 0: tile A (warps 0-3), 1: tile B (warps 4-7)
         const int row = tid & 127;        // TMEM lane == query row of the tile
-        const int qrow = it.q0[x] + row;
+        const int q0 = x ? it.q0b : it.q0a;
+        const int qrow = q0 + row;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + tmem_s(x);
         const uint32_t tO = tmem + lane_base + tmem_o(x);
@@ -427,7 +428,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         float l_run = 0.f;
         bool ok = true;
         for (int j = 0; j < n; ++j) {
-            if (!mbar_wait(bar(kSFull + x), j & 1, abort_flag)) {
+            // Waits that guard warp-collective tcgen05 instructions are made
+            // warp-uniform, so a timeout can never split a warp at one of them.
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(kSFull + x), j & 1, abort_flag))) {
                 ok = false;
                 break;
             }
@@ -446,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int src, row0;
             tile_of(it, j, src, row0);
             const bool full =
-                it.retr && ((src == 0 && row0 + kTileK <= p.len) || (src == 2 && row0 + kTileK <= it.q0[x]));
+                it.retr && ((src == 0 && row0 + kTileK <= p.len) || (src == 2 && row0 + kTileK <= q0));
             if (!full) {
 #pragma unroll
                 for (int w = 0; w < kTileK / 32; ++w) {
@@ -504,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kPFull + x));
         }
-        if (ok && mbar_wait(bar(kOFinal + x), 0, abort_flag)) {
+        if (__all_sync(0xffffffffu, ok && mbar_wait(bar(kOFinal + x), 0, abort_flag))) {
             tc_fence_after();
             const float inv = 1.f / l_run;
             bf16* orow = p.out + ((static_cast<int64_t>(it.b) * p.C + qrow) * p.Hq + it.head) * D;
