@@ -1,39 +1,42 @@
 // prefill.cu — mixed-head attention of one prefill chunk (DuoAttention
 // pre-filling), retrieval and streaming heads in one launch, on tcgen05.
 //
-// One CTA = one (batch, query head, pair of 128-query tiles) work item: tiles
-// A = queries [256t, 256t+128) and B = [256t+128, 256t+256) of the chunk share
-// every K/V tile the CTA loads. Retrieval items come first, heaviest (last
-// tile pair) first; streaming items fill in behind them.
+// One CTA = one (batch, query head, 128-query tile) work item. Retrieval items
+// come first, heaviest (last query tile) first; streaming items fill in behind.
 //
 // Key tiles of 128 keys are listed per item and fully masked tiles are never
-// listed (the list is the union of what A and B need):
+// listed:
 //   retrieval: cache tiles covering [0, len) of the retrieval pool, then chunk
-//              tiles 0 .. (B's diagonal tile);
+//              tiles 0 .. (the diagonal tile);
 //   streaming: the streaming-cache tiles holding the sinks (and the ring when
-//              the window of A's first query reaches below len), chunk tiles
+//              the window of the first query reaches below len), chunk tiles
 //              holding chunk-resident sinks, then the band tiles
-//              [first query of A - recent + 1, last query of B].
+//              [first query - recent + 1, last query].
 // Keys are masked element-wise by absolute position only on tiles that need it.
 //
-// Warp roles (384 threads, three warpgroups):
-//   warps 0-3  softmax of tile A: thread t owns query row t (TMEM lane t);
-//   warps 4-7  softmax of tile B, same lanes, other TMEM columns;
-//   warp 8     TMA producer: Q_A and Q_B once, then K/V tiles into 2-stage rings;
-//   warp 9     TMEM allocator and MMA issuer (one thread); warps 10-11 idle.
-// Registers: launched at 168 per thread; the third warpgroup gives back down
-// to 72 and the softmax warpgroups take 216 (2*128*216 + 128*72 = 384*168).
-// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
-// The softmax writes P (bf16 pairs) back into its S columns at +32 and the
-// PV product reads it from there (A operand in TMEM). MMAs issued by one
-// thread execute in order, so S_X(j+1) is written only after PV_X(j) read P_X(j).
-// MMA issue order per key tile j:
-//   PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1)
-// so the tensor core works on one tile while the other tile's softmax runs.
+// Warp roles (384 threads):
+//   warps 0-7  softmax, two threads per query row: warps w and w+4 read the
+//              same TMEM lanes (rows 32*(w%4) ..), warp w keys 0-63 of a tile
+//              and O columns [0, D/2), warp w+4 keys 64-127 and O [D/2, D);
+//              the two halves of a row agree on its running max through shared
+//              memory (one named barrier per warp pair and key tile);
+//   warp 8     TMA producer of Q and the K tiles (2-stage ring);
+//   warp 10    TMA producer of the V tiles (2-stage ring);
+//   warp 9     TMEM allocator and MMA issuer (one thread); warp 11 idle.
+// TMEM: S in two 128-column buffers [0,128) [128,256), O at [256, 256+D),
+// Q at [384, 384 + D/2) as bf16 pairs. The softmax warps copy Q there once, so
+// both products take their A operand from TMEM and read only K or V from shared
+// memory (an SS product of 128x128 tiles would need the shared-memory port's
+// full bandwidth).
+// Key tile j uses S buffer j&1, so the tensor core computes S(j+1) while the
+// softmax works on S(j). The softmax writes P (bf16 pairs) back into the S
+// buffer it read, at column +32 (keys 0-63 at +32, keys 64-127 at +64), and
+// the PV product takes it from there (A operand in TMEM). MMA issue order per
+// key tile j (one thread; tcgen05 MMAs run in issue order, so a later QK never
+// overwrites a P before the PV that reads it): PV(j), QK(j+2).
 // Softmax runs in the exp2 domain with a stale-max rule: O and the row sum are
 // rescaled only when the row max grows by more than 2^8 (exact: both stay
-// relative to the same stale max). A commit after QK_X(j+1) covers PV_X(j),
-// so O_X is stable when the softmax sees S_X(j+1).
+// relative to the same stale max).
 // All operand tiles in shared memory are 128-byte swizzled (TMA writes them,
 // the MMA reads them through descriptors). Every mbarrier wait is time-bounded;
 // on timeout the CTA records kErrPrefillWait and unwinds.
@@ -45,48 +48,52 @@ namespace duo {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kSoftmaxRegs = 216;
-constexpr int kControlRegs = 72;
-static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * 168, "register split exceeds the launch");
 constexpr int kTileBytesPerColBlock = kTileQ * 128;  // 128 rows x 64 bf16 (128 B)
 constexpr float kRescaleThreshold = 8.0f;             // log2 units: rescale when max grows by > 2^8
+constexpr int kHalf = kTileK / 2;                     // keys per softmax thread and tile
 
 template <int D>
 struct Layout {
     static constexpr int kColBlocks = D / 64;
     static constexpr int kTile = kColBlocks * kTileBytesPerColBlock;  // Q, K or V tile
-    static constexpr int kQA = 0;
-    static constexpr int kQB = kQA + kTile;
-    static constexpr int kK = kQB + kTile;      // 2 stages
+    static constexpr int kQ = 0;
+    static constexpr int kK = kQ + kTile;       // 2 stages
     static constexpr int kV = kK + 2 * kTile;   // 2 stages
     static constexpr int kBar = kV + 2 * kTile;
-    static constexpr int kMisc = kBar + 32 * 8;
+    // Pair exchange: maxima [tile parity][half][row], ok flags [parity][half][quarter],
+    // row sums [half][row].
+    static constexpr int kXchg = kBar + 32 * 8;
+    static constexpr int kMisc = kXchg + (2 * 2 * 128 + 2 * 2 * 4 + 2 * 128) * 4;
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
-enum Bar {
-    kQFull = 0,
-    kKFull = 1,    // +stage
-    kVFull = 3,    // +stage
-    kKEmpty = 5,   // +stage
-    kVEmpty = 7,   // +stage
-    kSFull = 9,    // +tile (A, B)
-    kPFull = 11,   // +tile
-    kOFinal = 13,  // +tile
-    kDrain = 15,
-};
+// mbarrier indices
+constexpr int kQFull = 0;
+constexpr int kKFull = 1;      // + stage
+constexpr int kVFull = 3;      // + stage
+constexpr int kKEmpty = 5;     // + stage
+constexpr int kVEmpty = 7;     // + stage
+constexpr int kSFull = 9;      // + S buffer
+constexpr int kPFull = 11;     // + S buffer (8 arrivals: one per softmax warp)
+constexpr int kODone = 13;     // one phase per PV
+constexpr int kOFinal = 14;    // one phase, after the last PV
+constexpr int kDrain = 15;
+constexpr int kQTmem = 16;     // Q copied into TMEM (8 arrivals: one per softmax warp)
+// Every barrier is waited with a phase parity, so none may complete two phases
+// beyond the one its waiter waits for: S and P barriers are per S buffer (P(j+2)
+// needs S(j+2), which needs PV(j) to have consumed P(j)) and the output waits
+// on a single-phase barrier.
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemP = 32;  // P of tile X at S_X + 32 (64 columns of bf16 pairs)
-
-__device__ __forceinline__ uint32_t tmem_s(int x) { return x ? 128u : 0u; }
-__device__ __forceinline__ uint32_t tmem_o(int x) { return x ? 384u : 256u; }
+constexpr uint32_t kTmemO = 256;
+constexpr uint32_t kTmemP = 32;  // P of a key tile at its S buffer + 32 (64 columns of bf16 pairs)
+constexpr uint32_t kTmemQ = 384; // Q tile as bf16 pairs, D/2 columns (A operand of QK)
 
 // What one work item attends to.
 struct Item {
-    int b, head, g, tp, retr, pool;
-    int q0a, q0b;  // first chunk row of tile A / B (scalars: no local memory)
+    int b, head, g, qt, retr, pool;
+    int q0;       // first chunk row of the query tile
     int n_cache;  // cache tiles
     int src_cache;
     int a;        // streaming: chunk tiles holding chunk-resident sinks
@@ -96,8 +103,7 @@ struct Item {
 
 __device__ __forceinline__ Item make_item(const PrefillParams& p) {
     Item it;
-    const int n_tp = (p.n_qt + 1) / 2;
-    const int n_retr_items = p.n_retr_q * p.B * n_tp;
+    const int n_retr_items = p.n_retr_q * p.B * p.n_qt;
     int idx = blockIdx.x;
     int nh, hbase;
     if (idx < n_retr_items) {
@@ -108,28 +114,26 @@ __device__ __forceinline__ Item make_item(const PrefillParams& p) {
         nh = p.Hq - p.n_retr_q;
         hbase = p.n_retr_q;
     }
-    it.tp = n_tp - 1 - idx / (nh * p.B);
+    it.qt = p.n_qt - 1 - idx / (nh * p.B);
     const int rem = idx % (nh * p.B);
     it.head = p.qhead[hbase + rem / p.B];
     it.b = rem % p.B;
     it.g = it.head / p.G;
     it.retr = p.heads.is_retr[it.g];
     it.pool = p.heads.pool_idx[it.g];
-    it.q0a = it.tp * 2 * kTileQ;
-    it.q0b = it.q0a + kTileQ;
-    const int qt_last = (2 * it.tp + 1 < p.n_qt) ? 2 * it.tp + 1 : 2 * it.tp;
+    it.q0 = it.qt * kTileQ;
     const int64_t L = p.len;
     if (it.retr) {
         it.src_cache = 0;
         it.n_cache = static_cast<int>((L + kTileK - 1) / kTileK);
         it.a = 0;
         it.b0 = 0;
-        it.n_tiles = it.n_cache + qt_last + 1;
+        it.n_tiles = it.n_cache + it.qt + 1;
     } else {
         it.src_cache = 1;
         int64_t slots = 0;
         if (L > 0) {
-            const bool band_in_cache = (L > p.S) && (it.q0a < p.R - 1);
+            const bool band_in_cache = (L > p.S) && (it.q0 < p.R - 1);
             slots = band_in_cache ? (L < p.W ? L : p.W) : (L < p.S ? L : p.S);
         }
         it.n_cache = static_cast<int>((slots + kTileK - 1) / kTileK);
@@ -137,13 +141,13 @@ __device__ __forceinline__ Item make_item(const PrefillParams& p) {
         if (L < p.S) {
             const int64_t sink_rows = (p.S - L < p.C) ? (p.S - L) : p.C;
             a = static_cast<int>((sink_rows + kTileK - 1) / kTileK);
-            if (a > qt_last + 1) a = qt_last + 1;
+            if (a > it.qt + 1) a = it.qt + 1;
         }
-        const int band_lo = it.q0a - p.R + 1 > 0 ? it.q0a - p.R + 1 : 0;
+        const int band_lo = it.q0 - p.R + 1 > 0 ? it.q0 - p.R + 1 : 0;
         const int tb = band_lo / kTileK;
         it.a = a;
         it.b0 = a > tb ? a : tb;
-        it.n_tiles = it.n_cache + a + (qt_last + 1 - it.b0);
+        it.n_tiles = it.n_cache + a + (it.qt + 1 - it.b0);
     }
     return it;
 }
@@ -234,6 +238,12 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
     return d;
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // D[tmem] (+)= A[tmem] * B[smem], kind::f16: the PV product with P held in TMEM.
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -245,6 +255,11 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         : "memory");
 }
 
+// Named barrier over the two warps (64 threads) that share one row quarter.
+__device__ __forceinline__ void pair_sync(int quarter) {
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps maps) {
@@ -253,10 +268,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw_addr = smem_u32(smem_raw);
     const uint32_t base = (raw_addr + 1023u) & ~1023u;
     uint8_t* const sbase = smem_raw + (base - raw_addr);
+    const uint32_t sQ = base + Lay::kQ;
     const uint32_t sK = base + Lay::kK;
     const uint32_t sV = base + Lay::kV;
-    auto sQ = [&](int x) { return base + (x ? Lay::kQB : Lay::kQA); };
     auto bar = [&](int i) { return base + Lay::kBar + 8u * i; };
+    volatile float* xchg = reinterpret_cast<volatile float*>(sbase + Lay::kXchg);
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sbase + Lay::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + Lay::kMisc + 4);
 
@@ -273,10 +289,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(kKEmpty + s), 1);
             mbar_init(bar(kVEmpty + s), 1);
             mbar_init(bar(kSFull + s), 1);
-            mbar_init(bar(kPFull + s), 4);
-            mbar_init(bar(kOFinal + s), 1);
+            mbar_init(bar(kPFull + s), 8);
         }
+        mbar_init(bar(kODone), 1);
+        mbar_init(bar(kOFinal), 1);
         mbar_init(bar(kDrain), 1);
+        mbar_init(bar(kQTmem), 8);
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -291,178 +309,195 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const int n = it.n_tiles;
 
-    // Each role's code stays inside the branch that sets its register budget.
-    if (warp >= 8) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
-    if (warp == 8) {
-        // ------------------------------------------------------------ TMA producer
+    if (warp == 8 || warp == 10) {
+        // ------------------------------------------------------------ TMA producers
+        // Warp 8 loads Q and the K tiles, warp 10 the V tiles: K runs ahead of V,
+        // gated only by the QK products that free its stages.
         if (lane == 0) {
-            tma_prefetch_desc(&maps.q);
-            mbar_arrive_expect_tx(bar(kQFull), 2 * Lay::kTile);
-            for (int x = 0; x < 2; ++x)
+            const bool is_k = warp == 8;
+            if (is_k) {
+                tma_prefetch_desc(&maps.q);
+                mbar_arrive_expect_tx(bar(kQFull), Lay::kTile);
                 for (int kb = 0; kb < Lay::kColBlocks; ++kb)
-                    tma_load_4d(sQ(x) + kb * kTileBytesPerColBlock, &maps.q, bar(kQFull), kb * 64, it.head, x ? it.q0b : it.q0a,
-                                it.b);
-            int issued = 0;
+                    tma_load_4d(sQ + kb * kTileBytesPerColBlock, &maps.q, bar(kQFull), kb * 64, it.head, it.q0, it.b);
+            }
+            const uint32_t ring = is_k ? sK : sV;
+            const int full = is_k ? kKFull : kVFull;
+            const int empty = is_k ? kKEmpty : kVEmpty;
+            int issued = 0;  // tiles whose load was issued
             for (int j = 0; j < n; ++j) {
                 const int st = j & 1;
-                const uint32_t use = j >> 1;
                 int src, row0;
                 tile_of(it, j, src, row0);
-                const CUtensorMap* mk = src == 0 ? &maps.rk : (src == 1 ? &maps.sk : &maps.k);
-                const CUtensorMap* mv = src == 0 ? &maps.rv : (src == 1 ? &maps.sv : &maps.v);
+                const CUtensorMap* m =
+                    is_k ? (src == 0 ? &maps.rk : (src == 1 ? &maps.sk : &maps.k))
+                         : (src == 0 ? &maps.rv : (src == 1 ? &maps.sv : &maps.v));
                 const int zpool = it.pool * p.B + it.b;
-                if (j >= 2 && !mbar_wait(bar(kKEmpty + st), (use - 1) & 1, abort_flag)) {
+                if (j >= 2 && !mbar_wait(bar(empty + st), ((j >> 1) - 1) & 1, abort_flag)) {
                     record_abort(p.err, abort_flag);
                     break;
                 }
-                mbar_arrive_expect_tx(bar(kKFull + st), Lay::kTile);
+                mbar_arrive_expect_tx(bar(full + st), Lay::kTile);
                 for (int kb = 0; kb < Lay::kColBlocks; ++kb) {
-                    const uint32_t dst = sK + st * Lay::kTile + kb * kTileBytesPerColBlock;
-                    if (src == 2) tma_load_4d(dst, mk, bar(kKFull + st), kb * 64, it.g, row0, it.b);
-                    else tma_load_3d(dst, mk, bar(kKFull + st), kb * 64, row0, zpool);
+                    const uint32_t dst = ring + st * Lay::kTile + kb * kTileBytesPerColBlock;
+                    if (src == 2) tma_load_4d(dst, m, bar(full + st), kb * 64, it.g, row0, it.b);
+                    else tma_load_3d(dst, m, bar(full + st), kb * 64, row0, zpool);
                 }
-                if (j >= 2 && !mbar_wait(bar(kVEmpty + st), (use - 1) & 1, abort_flag)) {
-                    record_abort(p.err, abort_flag);
-                    issued = 2 * j + 1;
-                    break;
-                }
-                mbar_arrive_expect_tx(bar(kVFull + st), Lay::kTile);
-                for (int kb = 0; kb < Lay::kColBlocks; ++kb) {
-                    const uint32_t dst = sV + st * Lay::kTile + kb * kTileBytesPerColBlock;
-                    if (src == 2) tma_load_4d(dst, mv, bar(kVFull + st), kb * 64, it.g, row0, it.b);
-                    else tma_load_3d(dst, mv, bar(kVFull + st), kb * 64, row0, zpool);
-                }
-                issued = 2 * j + 2;
+                issued = j + 1;
             }
             // Let every load this thread issued land before the CTA can exit.
-            const int nk = (issued + 1) / 2, nv = issued / 2;  // tiles with K / V issued
-            for (int j = (nk > 2 ? nk - 2 : 0); j < nk; ++j)
-                mbar_wait(bar(kKFull + (j & 1)), (j >> 1) & 1, nullptr);
-            for (int j = (nv > 2 ? nv - 2 : 0); j < nv; ++j)
-                mbar_wait(bar(kVFull + (j & 1)), (j >> 1) & 1, nullptr);
+            for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
+                mbar_wait(bar(full + (j & 1)), (j >> 1) & 1, nullptr);
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kTileK, 0, 0);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-            auto qk = [&](int x, int j) {
-                const uint32_t kt = sK + (j & 1) * Lay::kTile;
-                const uint32_t qt = sQ(x);
+            // S(j) = Q K(j)^T into S buffer j&1.
+            auto qk = [&](int j) -> bool {
+                const int st = j & 1;
+                if (!mbar_wait(bar(kKFull + st), (j >> 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t kt = sK + st * Lay::kTile;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kTileBytesPerColBlock + (kk & 3) * 32;
-                    tc_mma_ss(tmem + tmem_s(x), smem_desc_sw128(qt + off, 16, 1024),
-                              smem_desc_sw128(kt + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                    tc_mma_ts(tmem + st * kTileK, tmem + kTmemQ + kk * 8, smem_desc_sw128(kt + off, 16, 1024),
+                              idesc_qk, kk > 0 ? 1u : 0u);
                 }
-                tc_commit(bar(kSFull + x));
+                tc_commit(bar(kSFull + st));
+                tc_commit(bar(kKEmpty + st));
+                return true;
             };
-            auto pv = [&](int x, int j) {
-                const uint32_t vt = sV + (j & 1) * Lay::kTile;
+            bool ok = mbar_wait(bar(kQTmem), 0, abort_flag);
+            if (ok) tc_fence_after();
+            for (int j = 0; ok && j < 2 && j < n; ++j) ok = qk(j);
+            for (int j = 0; ok && j < n; ++j) {
+                const int st = j & 1;
+                if (!mbar_wait(bar(kVFull + st), (j >> 1) & 1, abort_flag) ||
+                    !mbar_wait(bar(kPFull + st), (j >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                // O += P(j) V(j), P(j) in TMEM at S buffer j&1 + kTmemP.
+                const uint32_t vt = sV + st * Lay::kTile;
 #pragma unroll
                 for (int kk = 0; kk < kTileK / 16; ++kk) {
                     const uint64_t bd = smem_desc_sw128(vt + kk * 2048, kTileBytesPerColBlock, 1024);
-                    tc_mma_ts(tmem + tmem_o(x), tmem + tmem_s(x) + kTmemP + kk * 8, bd, idesc_pv,
+                    tc_mma_ts(tmem + kTmemO, tmem + st * kTileK + kTmemP + kk * 8, bd, idesc_pv,
                               (j > 0 || kk > 0) ? 1u : 0u);
                 }
-            };
-            bool ok = mbar_wait(bar(kQFull), 0, abort_flag) && mbar_wait(bar(kKFull + 0), 0, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                qk(0, 0);
-                qk(1, 0);
-                tc_commit(bar(kKEmpty + 0));
-            }
-            for (int j = 0; ok && j < n; ++j) {
-                const int st = j & 1;
-                const bool more = j + 1 < n;
-                if (!mbar_wait(bar(kVFull + st), (j >> 1) & 1, abort_flag) ||
-                    !mbar_wait(bar(kPFull + 0), j & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                pv(0, j);
-                if (!more) tc_commit(bar(kOFinal + 0));
-                if (more) {
-                    if (!mbar_wait(bar(kKFull + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    qk(0, j + 1);
-                }
-                if (!mbar_wait(bar(kPFull + 1), j & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                pv(1, j);
+                tc_commit(bar(kODone));
+                if (j + 1 == n) tc_commit(bar(kOFinal));
                 tc_commit(bar(kVEmpty + st));
-                if (!more) tc_commit(bar(kOFinal + 1));
-                if (more) {
-                    qk(1, j + 1);
-                    tc_commit(bar(kKEmpty + ((j + 1) & 1)));
-                }
+                if (j + 2 < n) ok = qk(j + 2);
             }
             if (!ok) record_abort(p.err, abort_flag);
             // Drain: every MMA issued above completes before TMEM is released.
             tc_commit(bar(kDrain));
             mbar_wait(bar(kDrain), 0, nullptr);
         }
-    }
-    } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+    } else if (warp < 8) {
         // ------------------------------------------------------------ softmax warps
-        const int x = warp >> 2;          // 0: tile A (warps 0-3), 1: tile B (warps 4-7)
-        const int row = tid & 127;        // TMEM lane == query row of the tile
-        const int q0 = x ? it.q0b : it.q0a;
-        const int qrow = q0 + row;
-        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_base + tmem_s(x);
-        const uint32_t tO = tmem + lane_base + tmem_o(x);
+        const int quarter = warp & 3;  // TMEM lanes 32*quarter .. (query rows)
+        const int h = warp >> 2;       // key half of every tile, and half of O's columns
+        const int row = quarter * 32 + lane;
+        const int qrow = it.q0 + row;
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t tO = tmem + lane_base + kTmemO + h * (D / 2);
         const int64_t ring_last_r = (p.len > p.S) ? (p.len - 1 - p.S) % p.R : 0;
         const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
+        // Exchange area: [tile parity][half][row] maxima, then ok flags per warp.
+        volatile float* xmax = xchg;
+        volatile int* xok = reinterpret_cast<volatile int*>(xchg + 2 * 2 * 128);
+        volatile float* xsum = xchg + 2 * 2 * 128 + 2 * 2 * 4;
         float m_run = -INFINITY;
-        float l_run = 0.f;
+        float l_run = 0.f;  // this thread's half of the row sum
         bool ok = true;
+        // Q row -> TMEM (lane = row, bf16 pairs along D): QK then reads only K from
+        // shared memory. Each half copies D/2 elements of its row out of the
+        // 128-byte-swizzled TMA tile (16-byte chunk c of row r sits at c ^ (r % 8)).
+        if (__all_sync(0xffffffffu, mbar_wait(bar(kQFull), 0, abort_flag))) {
+            constexpr int kChunks = D / 16;  // 16-byte chunks per half row
+            uint32_t qv[kChunks * 4];
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+                const int e0 = h * (D / 2) + c * 8;
+                const uint32_t addr = sQ + (e0 / 64) * kTileBytesPerColBlock + row * 128 +
+                                      ((((e0 % 64) / 8) ^ (row & 7)) * 16);
+                const uint4 v4 = lds128(addr);
+                qv[c * 4 + 0] = v4.x;
+                qv[c * 4 + 1] = v4.y;
+                qv[c * 4 + 2] = v4.z;
+                qv[c * 4 + 3] = v4.w;
+            }
+            const uint32_t tq = tmem + lane_base + kTmemQ + h * (D / 4);
+            if constexpr (D == 128) tmem_st32(tq, qv);
+            else tmem_st16(tq, qv);
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kQTmem));
+        } else {
+            ok = false;
+            record_abort(p.err, abort_flag);
+        }
         for (int j = 0; j < n; ++j) {
-            // Waits that guard warp-collective tcgen05 instructions are made
-            // warp-uniform, so a timeout can never split a warp at one of them.
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(kSFull + x), j & 1, abort_flag))) {
+            const int buf = j & 1;
+            const uint32_t tS = tmem + lane_base + buf * kTileK;
+            // Waits that guard warp-collective tcgen05 instructions are warp-uniform;
+            // the two warps of a pair also leave the loop together (the named barrier
+            // below has no timeout).
+            const bool ok_s = ok && __all_sync(0xffffffffu, mbar_wait(bar(kSFull + buf), (j >> 1) & 1, abort_flag));
+            float s[kHalf];
+            float mh = -INFINITY;
+            if (ok_s) {
+                tc_fence_after();
+                uint32_t r[2][32];
+                tmem_ld32(tS + h * kHalf, r[0]);
+                tmem_ld32(tS + h * kHalf + 32, r[1]);
+                tc_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[c][i]);
+                int src, row0;
+                tile_of(it, j, src, row0);
+                const bool full =
+                    it.retr && ((src == 0 && row0 + kTileK <= p.len) || (src == 2 && row0 + kTileK <= it.q0));
+                if (!full) {
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        const uint32_t bits = visible_bits(p, it.retr, src, row0, 2 * h + w, qrow, ring_last_r);
+#pragma unroll
+                        for (int k = 0; k < 32; ++k)
+                            if (!((bits >> k) & 1u)) s[w * 32 + k] = -INFINITY;
+                    }
+                }
+                float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+                static_assert(kHalf % 8 == 0, "the max loop covers exactly [0, kHalf)");
+#pragma unroll
+                for (int i = 0; i < kHalf; i += 8) {
+                    m0 = fmax3(m0, s[i], s[i + 1]);
+                    m1 = fmax3(m1, s[i + 2], s[i + 3]);
+                    m2 = fmax3(m2, s[i + 4], s[i + 5]);
+                    m3 = fmax3(m3, s[i + 6], s[i + 7]);
+                }
+                mh = fmax3(fmaxf(m0, m1), m2, m3);
+            }
+            xmax[(buf * 2 + h) * 128 + row] = mh;
+            if (lane == 0) xok[(buf * 2 + h) * 4 + quarter] = ok_s ? 1 : 0;
+            pair_sync(quarter);
+            const float mo = xmax[(buf * 2 + (1 - h)) * 128 + row];
+            const bool ok_o = xok[(buf * 2 + (1 - h)) * 4 + quarter] != 0;
+            if (!ok_s || !ok_o) {
                 ok = false;
                 break;
             }
-            tc_fence_after();
-            float s[kTileK];
-            {
-                uint32_t r[32];
-#pragma unroll
-                for (int c = 0; c < kTileK / 32; ++c) {
-                    tmem_ld32(tS + c * 32, r);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
-                }
-            }
-            int src, row0;
-            tile_of(it, j, src, row0);
-            const bool full =
-                it.retr && ((src == 0 && row0 + kTileK <= p.len) || (src == 2 && row0 + kTileK <= q0));
-            if (!full) {
-#pragma unroll
-                for (int w = 0; w < kTileK / 32; ++w) {
-                    const uint32_t bits = visible_bits(p, it.retr, src, row0, w, qrow, ring_last_r);
-#pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        if (!((bits >> k) & 1u)) s[w * 32 + k] = -INFINITY;
-                }
-            }
-            float mt = fmaxf(s[0], s[1]);
-#pragma unroll
-            for (int i = 2; i < kTileK; ++i) mt = fmaxf(mt, s[i]);
-            mt *= p.scale_log2;
+            // Both halves of the row see the same max and take the same decision.
+            const float mt = fmaxf(mh, mo) * p.scale_log2;
             float factor = 1.f;
             if (mt > m_run + kRescaleThreshold) {  // also taken when m_run is -inf and mt finite
                 factor = fast_exp2(m_run - mt);
@@ -470,50 +505,57 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
             const uint64_t negm = f2pack(-m_use, -m_use);
-
-            // O_X is stable here: the commit behind S_X(j) covered PV_X(j-1).
-            if (j >= 1 && __any_sync(0xffffffffu, factor != 1.f)) {
-                uint32_t r[32];
+            uint64_t acc2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
+            uint32_t pk[kHalf / 2];
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    tmem_ld32(tO + c * 32, r);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * factor);
-                    tmem_st32(tO + c * 32, r);
-                }
-            }
-            // P = exp2(s * scale - m) as bf16 pairs, stored into TMEM 64 keys at a time.
-            uint64_t acc2 = f2pack(0.f, 0.f);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 64; i += 2) {
-                    float e0, e1;
-                    f2unpack(ffma2(f2pack(s[h * 64 + i], s[h * 64 + i + 1]), scale2, negm), e0, e1);
-                    const float p0 = fast_exp2(e0);
-                    const float p1 = fast_exp2(e1);
-                    acc2 = fadd2(acc2, f2pack(p0, p1));
-                    pk[i / 2] = pack_bf16x2(p0, p1);
-                }
-                tmem_st32(tS + kTmemP + h * 32, pk);
+            for (int i = 0; i < kHalf; i += 2) {
+                float e0, e1;
+                f2unpack(ffma2(f2pack(s[i], s[i + 1]), scale2, negm), e0, e1);
+                const float p0 = fast_exp2(e0);
+                const float p1 = fast_exp2(e1);
+                acc2[(i / 2) & 1] = fadd2(acc2[(i / 2) & 1], f2pack(p0, p1));
+                pk[i / 2] = pack_bf16x2(p0, p1);
             }
             float a0, a1;
-            f2unpack(acc2, a0, a1);
+            f2unpack(fadd2(acc2[0], acc2[1]), a0, a1);
             l_run = l_run * factor + (a0 + a1);
+            tmem_st32(tS + kTmemP + h * (kHalf / 2), pk);  // P of this half (S columns already read)
+            // O must be complete before it is rescaled: PV(j-1) is the last MMA that
+            // wrote it (kODone completes one phase per PV; the commit behind S(j)
+            // covered PV(j-2)). Each half rescales its own D/2 columns.
+            if (j >= 1 && __any_sync(0xffffffffu, factor != 1.f)) {
+                if (__all_sync(0xffffffffu, mbar_wait(bar(kODone), (j - 1) & 1, abort_flag))) {
+                    tc_fence_after();
+                    uint32_t r[32];
+#pragma unroll
+                    for (int c = 0; c < D / 64; ++c) {
+                        tmem_ld32(tO + c * 32, r);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * factor);
+                        tmem_st32(tO + c * 32, r);
+                    }
+                } else {
+                    ok = false;  // the pair leaves together at the next exchange
+                    record_abort(p.err, abort_flag);
+                }
+            }
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kPFull + x));
+            if (lane == 0) mbar_arrive(bar(kPFull + buf));
         }
-        if (__all_sync(0xffffffffu, ok && mbar_wait(bar(kOFinal + x), 0, abort_flag))) {
+        // Row sum of both halves, then the output: each half writes its D/2 columns.
+        xsum[h * 128 + row] = l_run;
+        pair_sync(quarter);
+        const float l_all = l_run + xsum[(1 - h) * 128 + row];
+        if (__all_sync(0xffffffffu, ok && mbar_wait(bar(kOFinal), 0, abort_flag))) {
             tc_fence_after();
-            const float inv = 1.f / l_run;
-            bf16* orow = p.out + ((static_cast<int64_t>(it.b) * p.C + qrow) * p.Hq + it.head) * D;
+            const float inv = 1.f / l_all;
+            bf16* orow = p.out + ((static_cast<int64_t>(it.b) * p.C + qrow) * p.Hq + it.head) * D + h * (D / 2);
             uint32_t r[32];
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < D / 64; ++c) {
                 tmem_ld32(tO + c * 32, r);
                 tc_wait_ld();
                 if (qrow < p.C) {
@@ -546,7 +588,7 @@ cudaError_t launch_d(const PrefillParams& p, const PrefillMaps& maps, cudaStream
     const int smem = Layout<128>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = static_cast<unsigned>(p.B * p.Hq * ((p.n_qt + 1) / 2));
+    const unsigned grid = static_cast<unsigned>(p.B * p.Hq * p.n_qt);
     prefill_kernel<D><<<grid, kThreads, smem, s>>>(p, maps);
     return cudaGetLastError();
 }
