@@ -101,6 +101,9 @@ def _ptr(x) -> Optional[int]:
 def _stream(stream) -> Optional[int]:
     if stream is None:
         import torch
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        if raw is not None:  # the current stream's handle without building a Stream object
+            return raw(torch.cuda.current_device())
         return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, int):
         return stream

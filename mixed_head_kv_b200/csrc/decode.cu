@@ -31,6 +31,10 @@ namespace {
 constexpr int kWarps = kDecodeThreads / 32;
 constexpr int kStages = 3;
 constexpr int kGroupRows = 4;  // row groups accumulated per register batch
+// Rows per warp hinted into L2 before the wait for the previous kernel (32 KB of
+// K and V at D = 128).
+template <int D>
+constexpr int64_t kPrefetchRows = 16384 / (D * 2);
 
 template <int D>
 struct Geom {
@@ -224,7 +228,6 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     float* sm_m = reinterpret_cast<float*>(smem);                 // [kWarps][G]
     float* sm_l = sm_m + kWarps * G;                              // [kWarps][G]
     float* sm_o = sm_l + kWarps * G;                              // [kWarps][G][D]
-    float* sm_w = sm_o + kWarps * G * D;                          // [G][kDecodeMaxSplits]
     int* sm_last = reinterpret_cast<int*>(smem + Gm::kBarOff + kWarps * kStages * 8);
 
     const int tid = threadIdx.x;
@@ -238,10 +241,6 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
         fence_barrier_init();
     }
     __syncwarp();
-    // Launched with programmatic stream serialization: everything above overlaps
-    // the previous kernel's tail; no global memory is touched before this wait.
-    grid_dependency_wait();
-    grid_launch_dependents();
 
     const int n_retr_items = p.B * p.n_retr * p.nsplit;
     const bool is_retr = static_cast<int>(blockIdx.x) < n_retr_items;
@@ -291,6 +290,26 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     const bf16* knew = p.k_new + (static_cast<int64_t>(b) * p.Hkv + g) * D;
     const bf16* vnew = p.v_new + (static_cast<int64_t>(b) * p.Hkv + g) * D;
 
+    // This warp's rows (contiguous, whole 4 KB blocks except at the end).
+    const int64_t n_rows = r1 - r0;
+    const int64_t per_warp = ((n_rows + kWarps - 1) / kWarps + Gm::BLK - 1) / Gm::BLK * Gm::BLK;
+    const int64_t w0 = r0 + warp * per_warp;
+    const int64_t w1 = (w0 + per_warp < r1) ? (w0 + per_warp) : r1;
+
+    // Launched with programmatic stream serialization: the CTA may start while
+    // the previous kernel of the stream drains. Before waiting for it, only hint
+    // the first rows of this warp into L2 (a prefetch reads no data into the CTA,
+    // and L2 stays coherent with the previous kernel's writes). Everything the
+    // kernel reads or writes comes after the wait.
+    if (lane == 0 && w0 < w1) {
+        const int64_t pre = (w1 - w0 < kPrefetchRows<D>) ? (w1 - w0) : kPrefetchRows<D>;
+        const uint32_t bytes = static_cast<uint32_t>(pre * D * 2);
+        bulk_prefetch_l2(kbase + w0 * D, bytes);
+        bulk_prefetch_l2(vbase + w0 * D, bytes);
+    }
+    grid_dependency_wait();
+    grid_launch_dependents();
+
     // Append the new token (D1): warp 1 copies it into its slot.
     if (owns_new && warp == 1) {
         if (lane < LPR) {
@@ -315,10 +334,6 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
 
     DecState<G> st;
     init_state(st);
-    const int64_t n_rows = r1 - r0;
-    const int64_t per_warp = ((n_rows + kWarps - 1) / kWarps + Gm::BLK - 1) / Gm::BLK * Gm::BLK;
-    const int64_t w0 = r0 + warp * per_warp;
-    const int64_t w1 = (w0 + per_warp < r1) ? (w0 + per_warp) : r1;
     bool ok = true;
     if (w0 < w1) ok = warp_stream<D, G>(st, qf, kbase, vbase, w0, w1, skip, ring, bars);
     if (!ok && lane == 0) atomicOr(p.err, kErrDecodeCopy);
@@ -381,64 +396,71 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     if (!*sm_last) return;
     __threadfence();
     // The partials of this (b, KV head) are contiguous: [nsplit][G][D] floats and
-    // [nsplit][G] log-sum-exps. Weights first, then a coalesced float4 pass in
-    // which each thread folds an independent subset of the splits.
+    // [nsplit][G] log-sum-exps. One coalesced float4 pass: each thread folds an
+    // independent subset of the splits with a running max (the log-sum-exp and
+    // the partial of a split are loaded together), then the subsets are combined.
     const int64_t item0 = (static_cast<int64_t>(b) * p.n_retr + ri) * p.nsplit;
     const int ns = p.nsplit;
-    for (int h = warp; h < G; h += kWarps) {
-        float M = -INFINITY;
-        for (int s = lane; s < ns; s += 32) {
-            const float x = __ldcg(p.part_lse + (item0 + s) * G + h);
-            sm_w[h * kDecodeMaxSplits + s] = x;
-            M = fmaxf(M, x);
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        float sum = 0.f;
-        for (int s = lane; s < ns; s += 32) {
-            const float w = fast_exp2(sm_w[h * kDecodeMaxSplits + s] - M);
-            sm_w[h * kDecodeMaxSplits + s] = w;
-            sum += w;
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        const float inv = 1.f / sum;
-        for (int s = lane; s < ns; s += 32) sm_w[h * kDecodeMaxSplits + s] *= inv;
-    }
-    __syncthreads();
     constexpr int kUnits = G * D / 4;  // float4 units of one split's partial
     constexpr int kRep = kUnits >= kDecodeThreads ? 1 : kDecodeThreads / kUnits;
-    float* sm_red = sm_w + G * kDecodeMaxSplits;  // [kRep][kUnits] float4
+    float4* sm_acc = reinterpret_cast<float4*>(smem);                 // [kRep][kUnits]
+    float* sm_mx = reinterpret_cast<float*>(sm_acc + kRep * kUnits);  // [kRep][kUnits]
+    float* sm_ls = sm_mx + kRep * kUnits;                             // [kRep][kUnits]
     const float4* po = reinterpret_cast<const float4*>(p.part_o + item0 * G * D);
+    const float* pl = p.part_lse + item0 * G;
+    __syncthreads();  // the per-warp merge arrays above are no longer read
     for (int u = tid % kUnits; u < kUnits; u += kDecodeThreads) {
         const int h = (u * 4) / D;
         const int rep = tid / kUnits;  // < kRep
+        float M = -INFINITY, Ls = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
+#pragma unroll 4
         for (int s = rep; s < ns; s += kRep) {
-            const float w = sm_w[h * kDecodeMaxSplits + s];
-            const float4 x = __ldcg(po + static_cast<int64_t>(s) * kUnits + u);
-            acc.x = fmaf(w, x.x, acc.x);
-            acc.y = fmaf(w, x.y, acc.y);
-            acc.z = fmaf(w, x.z, acc.z);
-            acc.w = fmaf(w, x.w, acc.w);
+            const float x = __ldcg(pl + static_cast<int64_t>(s) * G + h);
+            const float4 o = __ldcg(po + static_cast<int64_t>(s) * kUnits + u);
+            if (x > M) {  // every partial has a finite log-sum-exp
+                const float f = fast_exp2(M - x);  // 0 while M is -inf
+                Ls *= f;
+                acc.x *= f;
+                acc.y *= f;
+                acc.z *= f;
+                acc.w *= f;
+                M = x;
+            }
+            const float w = fast_exp2(x - M);
+            Ls += w;
+            acc.x = fmaf(w, o.x, acc.x);
+            acc.y = fmaf(w, o.y, acc.y);
+            acc.z = fmaf(w, o.z, acc.z);
+            acc.w = fmaf(w, o.w, acc.w);
         }
-        reinterpret_cast<float4*>(sm_red)[rep * kUnits + u] = acc;
+        sm_acc[rep * kUnits + u] = acc;
+        sm_mx[rep * kUnits + u] = M;
+        sm_ls[rep * kUnits + u] = Ls;
     }
     __syncthreads();
     for (int u = tid; u < kUnits; u += kDecodeThreads) {
-        float4 acc = reinterpret_cast<const float4*>(sm_red)[u];
-        for (int r = 1; r < kRep; ++r) {
-            const float4 x = reinterpret_cast<const float4*>(sm_red)[r * kUnits + u];
-            acc.x += x.x;
-            acc.y += x.y;
-            acc.z += x.z;
-            acc.w += x.w;
+        float M = -INFINITY;
+        for (int r = 0; r < kRep; ++r) M = fmaxf(M, sm_mx[r * kUnits + u]);
+        float Ls = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < kRep; ++r) {
+            const float mr = sm_mx[r * kUnits + u];
+            if (mr == -INFINITY) continue;  // this subset held no split
+            const float f = fast_exp2(mr - M);
+            const float4 x = sm_acc[r * kUnits + u];
+            Ls = fmaf(f, sm_ls[r * kUnits + u], Ls);
+            acc.x = fmaf(f, x.x, acc.x);
+            acc.y = fmaf(f, x.y, acc.y);
+            acc.z = fmaf(f, x.z, acc.z);
+            acc.w = fmaf(f, x.w, acc.w);
         }
+        const float inv = 1.f / Ls;
         const int h = (u * 4) / D;
         const int d = (u * 4) % D;
         bf16* o = p.out + (static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d;
-        *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        *reinterpret_cast<uint2*>(o) =
+            make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
     }
     if (tid == 0) p.counters[b * p.Hkv + g] = 0u;  // ready for the next step (stream-ordered)
 }
@@ -446,10 +468,11 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
 template <int D, int G>
 cudaError_t launch_dg(const DecodeParams& p, unsigned grid, cudaStream_t s) {
     constexpr int smem = Geom<D>::kSmem;
-    static_assert((kWarps * 2 * G + kWarps * G * D + G * kDecodeMaxSplits) * 4 + 16 * 2 * kDecodeThreads +
-                          16 * G * D / 4 <= Geom<D>::kRingBytes,
-                  "merge arrays must fit in the ring");
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    static_assert((kWarps * 2 * G + kWarps * G * D) * 4 <= Geom<D>::kRingBytes, "warp merge arrays fit in the ring");
+    static_assert((16 + 8) * (G * D / 4 >= kDecodeThreads ? G * D / 4 : kDecodeThreads) <= Geom<D>::kRingBytes,
+                  "split merge arrays fit in the ring");
+    static SmemLimitOnce limit;
+    cudaError_t e = limit.apply(reinterpret_cast<const void*>(&decode_kernel<D, G>), smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(decode_kernel<D, G>, dim3(grid), dim3(kDecodeThreads), smem, s, p);
 }

@@ -212,6 +212,33 @@ duo_status duo_cache_alloc(const duo_layout* layout, const uint8_t* is_retrieval
         delete c;
         return DUO_ERR_CUDA;
     }
+    // Decode parameters that do not change between steps, per layer.
+    c->decode_tmpl.assign(L.num_layers, DecodeParams{});
+    for (int32_t layer = 0; layer < L.num_layers; ++layer) {
+        DecodeParams& t = c->decode_tmpl[layer];
+        t.pools = c->pools;
+        t.part_o = c->part_o;
+        t.part_lse = c->part_lse;
+        t.counters = c->counters;
+        t.err = c->err;
+        t.max_len = L.max_len;
+        t.B = L.batch;
+        t.Hq = L.num_q_heads;
+        t.Hkv = L.num_kv_heads;
+        t.G = c->G;
+        t.D = L.head_dim;
+        t.S = L.sink;
+        t.R = L.recent;
+        t.W = c->W;
+        t.scale_log2 = c->scale * 1.4426950408889634f;
+        fill_heads(c, layer, &t.heads);
+        for (int g = 0; g < L.num_kv_heads; ++g) {
+            if (t.heads.is_retr[g]) t.retr_list[t.n_retr++] = static_cast<int16_t>(g);
+            else t.strm_list[t.n_strm++] = static_cast<int16_t>(g);
+        }
+    }
+    c->plan_key.assign(L.num_layers, -1);
+    c->plan_nsplit.assign(L.num_layers, 1);
     *out = c;
     return DUO_OK;
 }
@@ -343,35 +370,14 @@ duo_status duo_decode(duo_cache* c, int32_t layer, const void* q, const void* k_
     if (!q || !k_new || !v_new || !out) return DUO_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return DUO_ERR_ALIGNMENT;
     if (c->len[layer] + 1 > c->lay.max_len) return DUO_ERR_CAPACITY;
-    const duo_layout& L = c->lay;
-    DecodeParams p{};
+    DecodeParams p = c->decode_tmpl[layer];
     p.q = static_cast<const bf16*>(q);
     p.k_new = static_cast<const bf16*>(k_new);
     p.v_new = static_cast<const bf16*>(v_new);
     p.out = static_cast<bf16*>(out);
-    p.pools = c->pools;
-    p.part_o = c->part_o;
-    p.part_lse = c->part_lse;
-    p.counters = c->counters;
-    p.err = c->err;
     p.len = c->len[layer];
-    p.max_len = L.max_len;
-    p.B = L.batch;
-    p.Hq = L.num_q_heads;
-    p.Hkv = L.num_kv_heads;
-    p.G = c->G;
-    p.D = L.head_dim;
-    p.S = L.sink;
-    p.R = L.recent;
-    p.W = c->W;
-    p.scale_log2 = c->scale * 1.4426950408889634f;
-    fill_heads(c, layer, &p.heads);
-    for (int g = 0; g < L.num_kv_heads; ++g) {
-        if (p.heads.is_retr[g]) p.retr_list[p.n_retr++] = static_cast<int16_t>(g);
-        else p.strm_list[p.n_strm++] = static_cast<int16_t>(g);
-    }
     const int64_t rows = p.len + 1;
-    const int64_t nsplit = plan_decode_splits(L.batch, p.n_retr, p.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms);
+    const int64_t nsplit = decode_plan(c, layer, rows);
     p.split_rows = (rows + nsplit - 1) / nsplit;
     p.nsplit = static_cast<int32_t>((rows + p.split_rows - 1) / p.split_rows);
     if (launch_decode(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUO_ERR_CUDA;

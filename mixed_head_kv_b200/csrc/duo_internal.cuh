@@ -2,6 +2,7 @@
 // the host ABI (duo_abi.cu) and the kernels (append.cu, decode.cu, prefill.cu).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <vector>
 #include <cuda.h>
@@ -31,6 +32,21 @@ cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaSt
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, p);
 }
+
+// Sets a kernel's dynamic shared-memory limit once per device (the attribute
+// call costs host time on every launch otherwise). One instance per kernel.
+struct SmemLimitOnce {
+    std::atomic<uint64_t> done{0};
+    cudaError_t apply(const void* kernel, int smem) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+        const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+        if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return cudaSuccess;
+        const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_acq_rel);
+        return e;
+    }
+};
 
 // Per-layer KV-head map, passed by value: for every KV head its type and its
 // dense index in the retrieval pool or the streaming pool (over all layers).
@@ -168,4 +184,21 @@ struct duo_cache {
     uint32_t* counters = nullptr;
     uint32_t* err = nullptr;
     CUtensorMap map_rk{}, map_rv{}, map_sk{}, map_sv{};
+    std::vector<duo::DecodeParams> decode_tmpl;  // [layers] decode parameters fixed at alloc
+    std::vector<int64_t> plan_key;               // [layers] rows / 256 of the cached split plan
+    std::vector<int64_t> plan_nsplit;            // [layers] the plan's split count
 };
+
+// Split count for a decode step over `rows` keys of `layer`. The plan is kept
+// per layer and recomputed when rows / 256 changes: any split count is
+// correct, the plan only balances the launch.
+inline int64_t decode_plan(duo_cache* c, int32_t layer, int64_t rows) {
+    const int64_t key = rows >> 8;
+    if (c->plan_key[layer] != key) {
+        const duo::DecodeParams& t = c->decode_tmpl[layer];
+        c->plan_nsplit[layer] =
+            duo::plan_decode_splits(c->lay.batch, t.n_retr, t.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms);
+        c->plan_key[layer] = key;
+    }
+    return c->plan_nsplit[layer];
+}

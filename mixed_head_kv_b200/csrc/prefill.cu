@@ -586,7 +586,8 @@ cudaError_t launch_d(const PrefillParams& p, const PrefillMaps& maps, cudaStream
     // Same shared-memory request for every D: one CTA per SM, so a CTA never
     // waits on another for TMEM columns.
     const int smem = Layout<128>::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    static SmemLimitOnce limit;
+    cudaError_t e = limit.apply(reinterpret_cast<const void*>(&prefill_kernel<D>), smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = static_cast<unsigned>(p.B * p.Hq * p.n_qt);
     prefill_kernel<D><<<grid, kThreads, smem, s>>>(p, maps);
