@@ -513,6 +513,109 @@ def run_reference(args):
     print(json.dumps(res))
 
 
+# ----------------------------------------------------------------------------- secondary workloads
+def _fill_cache(duo, cache, w, layer, L, block=1 << 16):
+    for c0 in range(0, L, block):
+        n = min(block, L - c0)
+        kk, vv = workloads.tokens(w, layer, c0, n, device="cuda", which="kv")
+        cache.append(layer, kk, vv)
+
+
+def _time_decode_steps(duo, cache, w, layers, L, steps):
+    """Device time of `steps` decode steps (one launch per layer each), back to back."""
+    qkv = [workloads.tokens(w, l, L, steps, device="cuda") for l in layers]
+    ins = [[tuple(x[:, t].contiguous() for x in qkv[i]) for t in range(steps)] for i in range(len(layers))]
+    o = torch.empty_like(ins[0][0][0])
+    lib, sp = duo._lib, torch.cuda.current_stream().cuda_stream
+    res = []
+    for rep in range(2):  # the first pass warms up
+        for l in layers:
+            cache.set_length(l, L)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for t in range(steps):
+            for i, l in enumerate(layers):
+                q, k, v = ins[i][t]
+                if lib.duo_decode(cache.handle, l, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), sp):
+                    raise RuntimeError("decode failed")
+        e1.record()
+        torch.cuda.synchronize()
+        res.append(e0.elapsed_time(e1) * 1e-3 / steps)
+    if cache.error_flags():
+        raise RuntimeError("device error flag set")
+    return res[-1]
+
+
+def run_sweep(args):
+    """The other workloads of the benchmark definition (decode at 128K and 1M,
+    the MHA retrieval-ratio sweep): one JSON line each, device time only."""
+    torch.cuda.set_device(0)
+    import __graft_entry__
+    __graft_entry__.build()
+    import mixed_head_kv_b200 as duo
+    peaks = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    out = []
+
+    def emit(d):
+        print(json.dumps(d), flush=True)
+        out.append(d)
+
+    def decode_case(w, layers, steps):
+        L = w.context
+        masks = [workloads.retrieval_mask(w, l) for l in range(w.num_layers)]
+        cache = duo.DuoCache(w.num_layers, w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.sink, w.recent,
+                             L + steps + 1, [m for ms in masks for m in ms])
+        for l in layers:
+            _fill_cache(duo, cache, w, l, L)
+        t = _time_decode_steps(duo, cache, w, layers, L, steps)
+        byt = sum(statistics.fmean(decode_bytes(w, masks[l], L + s) for s in range(steps)) for l in layers)
+        emit({"workload": w.name, "phase": "decode", "batch": w.batch, "context": L, "layers": len(layers),
+              "us_per_step": t * 1e6, "tokens_per_s": w.batch / t, "kv_read_gbs": byt / t / 1e9,
+              "frac_of_measured_hbm": byt / t / 1e9 / hbm})
+        del cache
+        torch.cuda.empty_cache()
+
+    decode_case(workloads.LLAMA3_GQA, [0], 20)
+    for recent in (256, 1024):
+        for ratio in (0.0, 0.25, 0.5, 0.75, 1.0):
+            if recent == 1024 and ratio not in (0.0, 0.25):
+                continue
+            decode_case(workloads.mha_sweep(ratio, recent=recent), [0], 10)
+    decode_case(workloads.GQA_STACK_1M, list(range(workloads.GQA_STACK_1M.num_layers)), 4)
+
+    for recent, ratios in ((256, (0.0, 0.25, 0.5, 0.75, 1.0)), (1024, (0.0,))):
+        for ratio in ratios:
+            w = workloads.mha_sweep(ratio, recent=recent, prefill=True)
+            mask = workloads.retrieval_mask(w)
+            cache = duo.DuoCache(1, 1, 32, 32, 128, w.sink, w.recent, w.prefill_len, mask)
+            q, k, v = workloads.tokens(w, 0, 0, w.prefill_len, device="cuda")
+            chunks = [(p0, tuple(x[:, p0:p0 + w.chunk].contiguous() for x in (q, k, v)))
+                      for p0 in range(0, w.prefill_len, w.chunk)]
+            o = torch.empty_like(chunks[0][1][0])
+            times = []
+            for rep in range(2):
+                cache.set_length(0, 0)
+                ev = []
+                for p0, (qc, kc, vc) in chunks:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    cache.prefill(0, qc, kc, vc, o)
+                    e1.record()
+                    ev.append((e0, e1))
+                    cache.append(0, kc, vc)
+                torch.cuda.synchronize()
+                times.append(sum(a.elapsed_time(b) for a, b in ev) * 1e-3)
+            flop = sum(prefill_flops(w, mask, p0, w.chunk) for p0, _ in chunks)
+            emit({"workload": w.name, "phase": "prefill", "batch": 1, "context": w.prefill_len, "chunk": w.chunk,
+                  "ms_prefill_kernels": times[-1] * 1e3, "unmasked_tflops": flop / times[-1] / 1e12,
+                  "frac_of_measured_sustained": flop / times[-1] / 1e12 / peaks["bf16_tflops_sustained"]})
+            del cache, q, k, v, chunks
+            torch.cuda.empty_cache()
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -520,7 +623,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="duo", choices=["duo", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for the CPU baseline")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the other workloads (GQA decode at 128K and 1M, MHA ratio sweep) instead")
     args = ap.parse_args(argv)
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.warmup < 3 and args.impl != "reference":
         args.warmup = 3
     if args.impl == "reference":
