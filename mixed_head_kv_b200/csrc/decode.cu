@@ -51,10 +51,15 @@ struct Geom {
 
 template <int G>
 struct DecState {
-    float m[G];
+    float m[G];       // running max (log2 domain), stale by up to kDecodeRescale
     float l[G];
-    float o[G][8];
+    uint64_t o[G][4];  // output accumulators, packed fp32 pairs (elements 2i, 2i+1)
 };
+
+// The running max of a lane group is raised, and l and o rescaled, only when a
+// score exceeds it by more than 2^8: exact (l and o stay relative to the same
+// max), and the rescale is skipped for almost every row batch.
+constexpr float kDecodeRescale = 8.0f;
 
 template <int G>
 __device__ __forceinline__ void init_state(DecState<G>& st) {
@@ -63,31 +68,36 @@ __device__ __forceinline__ void init_state(DecState<G>& st) {
         st.m[h] = -INFINITY;
         st.l[h] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) st.o[h][e] = 0.f;
+        for (int i = 0; i < 4; ++i) st.o[h][i] = f2pack(0.f, 0.f);
     }
 }
 
+// Eight bf16 of a 16-byte slice as four packed fp32 pairs.
+__device__ __forceinline__ void bf16x8_to_f2(const uint4& x, uint64_t (&r)[4]) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r[i] = f2pack(bf16lo_to_f32(w[i]), bf16hi_to_f32(w[i]));
+}
+
 // Fold U row groups (this lane's 16-byte slices of K and V rows) into the state.
+// q2: this lane's 8 query elements of each head, pre-scaled into the exp2 domain.
 template <int D, int G, int U>
-__device__ __forceinline__ void accumulate(DecState<G>& st, const float (&qf)[G][8], const uint4 (&kx)[U],
+__device__ __forceinline__ void accumulate(DecState<G>& st, const uint64_t (&q2)[G][4], const uint4 (&kx)[U],
                                            const uint4 (&vx)[U], const bool (&valid)[U]) {
     constexpr int LPR = D / 8;
     float s[U][G];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-        const uint32_t w[4] = {kx[u].x, kx[u].y, kx[u].z, kx[u].w};
-        float kf[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            kf[2 * i] = bf16lo_to_f32(w[i]);
-            kf[2 * i + 1] = bf16hi_to_f32(w[i]);
-        }
+        uint64_t k2[4];
+        bf16x8_to_f2(kx[u], k2);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            float acc = 0.f;
+            uint64_t acc = f2pack(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc = fmaf(qf[h][e], kf[e], acc);
-            s[u][h] = acc;
+            for (int i = 0; i < 4; ++i) acc = ffma2(q2[h][i], k2[i], acc);
+            float lo, hi;
+            f2unpack(acc, lo, hi);
+            s[u][h] = lo + hi;
         }
     }
 #pragma unroll
@@ -105,34 +115,31 @@ __device__ __forceinline__ void accumulate(DecState<G>& st, const float (&qf)[G]
             for (int h = 0; h < G; ++h) s[u][h] = -INFINITY;
         }
     }
-    float vf[U][8];
+    uint64_t v2[U][4];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-        const uint32_t w[4] = {vx[u].x, vx[u].y, vx[u].z, vx[u].w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            vf[u][2 * i] = bf16lo_to_f32(w[i]);
-            vf[u][2 * i + 1] = bf16hi_to_f32(w[i]);
-        }
-    }
+    for (int u = 0; u < U; ++u) bf16x8_to_f2(vx[u], v2[u]);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         float mb = s[0][h];
 #pragma unroll
         for (int u = 1; u < U; ++u) mb = fmaxf(mb, s[u][h]);
-        const float mn = fmaxf(st.m[h], mb);
-        if (mn == -INFINITY) continue;  // nothing valid for this lane group yet
-        const float f = fast_exp2(st.m[h] - mn);  // 0 when the old max is -inf
-        st.m[h] = mn;
-        st.l[h] *= f;
+        if (mb > st.m[h] + kDecodeRescale) {  // also taken when m is -inf and mb finite
+            const float f = fast_exp2(st.m[h] - mb);  // 0 when the old max is -inf
+            st.m[h] = mb;
+            st.l[h] *= f;
+            const uint64_t f2 = f2pack(f, f);
+            const uint64_t z2 = f2pack(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) st.o[h][e] *= f;
+            for (int i = 0; i < 4; ++i) st.o[h][i] = ffma2(st.o[h][i], f2, z2);
+        }
+        if (st.m[h] == -INFINITY) continue;  // nothing valid for this lane group yet
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const float pu = fast_exp2(s[u][h] - mn);
+            const float pu = fast_exp2(s[u][h] - st.m[h]);
             st.l[h] += pu;
+            const uint64_t p2 = f2pack(pu, pu);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) st.o[h][e] = fmaf(pu, vf[u][e], st.o[h][e]);
+            for (int i = 0; i < 4; ++i) st.o[h][i] = ffma2(p2, v2[u][i], st.o[h][i]);
         }
     }
 }
@@ -149,10 +156,13 @@ __device__ __forceinline__ void merge_lanes(DecState<G>& st, int off) {
         const float f1 = fast_exp2(st.m[h] - ms);
         const float f2 = fast_exp2(m2 - ms);
         st.l[h] = st.l[h] * f1 + l2 * f2;
+        const uint64_t f1p = f2pack(f1, f1);
+        const uint64_t f2p = f2pack(f2, f2);
+        const uint64_t z2 = f2pack(0.f, 0.f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float o2 = __shfl_xor_sync(0xffffffffu, st.o[h][e], off);
-            st.o[h][e] = st.o[h][e] * f1 + o2 * f2;
+        for (int i = 0; i < 4; ++i) {
+            const uint64_t o2 = __shfl_xor_sync(0xffffffffu, st.o[h][i], off);
+            st.o[h][i] = ffma2(o2, f2p, ffma2(st.o[h][i], f1p, z2));
         }
         st.m[h] = mn;
     }
@@ -161,7 +171,7 @@ __device__ __forceinline__ void merge_lanes(DecState<G>& st, int off) {
 // Stream rows [r0, r1) (except `skip`) of one head through this warp's ring.
 // Returns false if a copy did not complete within the wait limit.
 template <int D, int G>
-__device__ bool warp_stream(DecState<G>& st, const float (&qf)[G][8], const bf16* kbase, const bf16* vbase,
+__device__ bool warp_stream(DecState<G>& st, const uint64_t (&q2)[G][4], const bf16* kbase, const bf16* vbase,
                             int64_t r0, int64_t r1, int64_t skip, uint32_t ring, uint32_t bars) {
     using Gm = Geom<D>;
     const int lane = threadIdx.x & 31;
@@ -208,7 +218,7 @@ __device__ bool warp_stream(DecState<G>& st, const float (&qf)[G][8], const bf16
                 kx[u] = valid[u] ? lds128(kst + off) : make_uint4(0, 0, 0, 0);
                 vx[u] = valid[u] ? lds128(vst + off) : make_uint4(0, 0, 0, 0);
             }
-            accumulate<D, G, kGroupRows>(st, qf, kx, vx, valid);
+            accumulate<D, G, kGroupRows>(st, q2, kx, vx, valid);
         }
         __syncwarp();
         if (lane == 0 && i + kStages < nblk) {
@@ -320,28 +330,26 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     }
 
     // Queries of the group, pre-scaled into the exp2 domain.
-    float qf[G][8];
+    uint64_t q2[G][4];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         const uint4 qx = ld_nc_v4(p.q + (static_cast<int64_t>(b) * p.Hq + g * G + h) * D + sub * 8);
         const uint32_t w[4] = {qx.x, qx.y, qx.z, qx.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            qf[h][2 * i] = bf16lo_to_f32(w[i]) * p.scale_log2;
-            qf[h][2 * i + 1] = bf16hi_to_f32(w[i]) * p.scale_log2;
-        }
+        for (int i = 0; i < 4; ++i)
+            q2[h][i] = f2pack(bf16lo_to_f32(w[i]) * p.scale_log2, bf16hi_to_f32(w[i]) * p.scale_log2);
     }
 
     DecState<G> st;
     init_state(st);
     bool ok = true;
-    if (w0 < w1) ok = warp_stream<D, G>(st, qf, kbase, vbase, w0, w1, skip, ring, bars);
+    if (w0 < w1) ok = warp_stream<D, G>(st, q2, kbase, vbase, w0, w1, skip, ring, bars);
     if (!ok && lane == 0) atomicOr(p.err, kErrDecodeCopy);
     if (owns_new && warp == 0) {
         uint4 kx[1] = {ld_nc_v4(knew + sub * 8)};
         uint4 vx[1] = {ld_nc_v4(vnew + sub * 8)};
         bool valid[1] = {lane < LPR};
-        accumulate<D, G, 1>(st, qf, kx, vx, valid);
+        accumulate<D, G, 1>(st, q2, kx, vx, valid);
     }
 
     // Merge the row groups of the warp, then the warps.
@@ -356,7 +364,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
                 sm_l[warp * G + h] = st.l[h];
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) sm_o[(warp * G + h) * D + sub * 8 + e] = st.o[h][e];
+            for (int i = 0; i < 4; ++i) {
+                float lo, hi;
+                f2unpack(st.o[h][i], lo, hi);
+                sm_o[(warp * G + h) * D + sub * 8 + 2 * i] = lo;
+                sm_o[(warp * G + h) * D + sub * 8 + 2 * i + 1] = hi;
+            }
         }
     }
     __syncthreads();
