@@ -16,24 +16,23 @@
 //
 // Warp roles (384 threads):
 //   warps 0-7  softmax, two threads per query row: warps w and w+4 read the
-//              same TMEM lanes (rows 32*(w%4) ..), warp w keys 0-63 of a tile
-//              and O columns [0, D/2), warp w+4 keys 64-127 and O [D/2, D);
-//              the two halves of a row agree on its running max through shared
-//              memory (one named barrier per warp pair and key tile);
+//              same TMEM lanes (rows 32*(w%4) ..); warp w takes keys 0-63 of
+//              every tile, warp w+4 keys 64-127. Each half keeps its own running
+//              max, row sum and O accumulator, so the halves never wait for each
+//              other inside the key loop; the epilogue combines them with
+//              log-sum-exp weights;
 //   warp 8     TMA producer of Q and the K tiles (2-stage ring);
 //   warp 10    TMA producer of the V tiles (2-stage ring);
 //   warp 9     TMEM allocator and MMA issuer (one thread); warp 11 idle.
-// TMEM: S in two 128-column buffers [0,128) [128,256), O at [256, 256+D),
-// Q at [384, 384 + D/2) as bf16 pairs. The softmax warps copy Q there once, so
-// both products take their A operand from TMEM and read only K or V from shared
-// memory (an SS product of 128x128 tiles would need the shared-memory port's
-// full bandwidth).
+// TMEM (512 columns): S in two 128-column buffers [0,128) [128,256), then O of
+// key half 0 at [256, 256+D) and of key half 1 at [256+D, 256+2D).
 // Key tile j uses S buffer j&1, so the tensor core computes S(j+1) while the
-// softmax works on S(j). The softmax writes P (bf16 pairs) back into the S
-// buffer it read, at column +32 (keys 0-63 at +32, keys 64-127 at +64), and
-// the PV product takes it from there (A operand in TMEM). MMA issue order per
-// key tile j (one thread; tcgen05 MMAs run in issue order, so a later QK never
-// overwrites a P before the PV that reads it): PV(j), QK(j+2).
+// softmax works on S(j). Each half writes its P (bf16 pairs) back into the S
+// buffer it read, at column +32 (keys 0-63) or +64 (keys 64-127), and the PV
+// product of that half (A operand in TMEM, four K=16 steps) accumulates into
+// its own O as soon as its four warps are done. MMA issue order per key tile j
+// (one thread; tcgen05 MMAs run in issue order, so a later QK never overwrites
+// a P before the PV that reads it): PV_0(j), PV_1(j), QK(j+2).
 // Softmax runs in the exp2 domain with a stale-max rule: O and the row sum are
 // rescaled only when the row max grows by more than 2^8 (exact: both stay
 // relative to the same stale max).
@@ -75,20 +74,19 @@ constexpr int kVFull = 3;      // + stage
 constexpr int kKEmpty = 5;     // + stage
 constexpr int kVEmpty = 7;     // + stage
 constexpr int kSFull = 9;      // + S buffer
-constexpr int kPFull = 11;     // + S buffer (8 arrivals: one per softmax warp)
-constexpr int kODone = 13;     // one phase per PV
-constexpr int kOFinal = 14;    // one phase, after the last PV
-constexpr int kDrain = 15;
-constexpr int kQTmem = 16;     // Q copied into TMEM (8 arrivals: one per softmax warp)
+constexpr int kP0Full = 11;    // + S buffer: P of keys 0-63 written (4 arrivals: warps 0-3)
+constexpr int kP1Full = 13;    // + S buffer: P of keys 64-127 written (4 arrivals: warps 4-7)
+constexpr int kODone = 15;     // one phase per key tile (both PV halves)
+constexpr int kOFinal = 16;    // one phase, after the last PV
+constexpr int kDrain = 17;
 // Every barrier is waited with a phase parity, so none may complete two phases
 // beyond the one its waiter waits for: S and P barriers are per S buffer (P(j+2)
-// needs S(j+2), which needs PV(j) to have consumed P(j)) and the output waits
-// on a single-phase barrier.
+// needs S(j+2), which needs both PV halves of tile j to have consumed P(j)) and
+// the output waits on a single-phase barrier.
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;
-constexpr uint32_t kTmemP = 32;  // P of a key tile at its S buffer + 32 (64 columns of bf16 pairs)
-constexpr uint32_t kTmemQ = 384; // Q tile as bf16 pairs, D/2 columns (A operand of QK)
+constexpr uint32_t kTmemO = 256;  // O of key half h at kTmemO + h * D
+constexpr uint32_t kTmemP = 32;   // P of a key tile at its S buffer + 32 (64 columns of bf16 pairs)
 
 // What one work item attends to.
 struct Item {
@@ -269,12 +267,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(kKEmpty + s), 1);
             mbar_init(bar(kVEmpty + s), 1);
             mbar_init(bar(kSFull + s), 1);
-            mbar_init(bar(kPFull + s), 8);
+            mbar_init(bar(kP0Full + s), 4);
+            mbar_init(bar(kP1Full + s), 4);
         }
         mbar_init(bar(kODone), 1);
         mbar_init(bar(kOFinal), 1);
         mbar_init(bar(kDrain), 1);
-        mbar_init(bar(kQTmem), 8);
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -343,32 +341,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kTileBytesPerColBlock + (kk & 3) * 32;
-                    tc_mma_ts(tmem + st * kTileK, tmem + kTmemQ + kk * 8, smem_desc_sw128(kt + off, 16, 1024),
-                              idesc_qk, kk > 0 ? 1u : 0u);
+                    tc_mma_ss(tmem + st * kTileK, smem_desc_sw128(sQ + off, 16, 1024),
+                              smem_desc_sw128(kt + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
                 }
                 tc_commit(bar(kSFull + st));
                 tc_commit(bar(kKEmpty + st));
                 return true;
             };
-            bool ok = mbar_wait(bar(kQTmem), 0, abort_flag);
-            if (ok) tc_fence_after();
+            bool ok = mbar_wait(bar(kQFull), 0, abort_flag);
             for (int j = 0; ok && j < 2 && j < n; ++j) ok = qk(j);
             for (int j = 0; ok && j < n; ++j) {
                 const int st = j & 1;
-                if (!mbar_wait(bar(kVFull + st), (j >> 1) & 1, abort_flag) ||
-                    !mbar_wait(bar(kPFull + st), (j >> 1) & 1, abort_flag)) {
+                if (!mbar_wait(bar(kVFull + st), (j >> 1) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                // O += P(j) V(j), P(j) in TMEM at S buffer j&1 + kTmemP.
+                // O_h += P_h(j) V_h(j) for the two key halves, each as soon as its
+                // four softmax warps have written P_h (in TMEM at S buffer j&1 + kTmemP).
                 const uint32_t vt = sV + st * Lay::kTile;
+                for (int half = 0; ok && half < 2; ++half) {
+                    if (!mbar_wait(bar((half ? kP1Full : kP0Full) + st), (j >> 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < kTileK / 16; ++kk) {
-                    const uint64_t bd = smem_desc_sw128(vt + kk * 2048, kTileBytesPerColBlock, 1024);
-                    tc_mma_ts(tmem + kTmemO, tmem + st * kTileK + kTmemP + kk * 8, bd, idesc_pv,
-                              (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const int kk = half * 4 + k4;
+                        const uint64_t bd = smem_desc_sw128(vt + kk * 2048, kTileBytesPerColBlock, 1024);
+                        tc_mma_ts(tmem + kTmemO + half * D, tmem + st * kTileK + kTmemP + kk * 8, bd, idesc_pv,
+                                  (j > 0 || k4 > 0) ? 1u : 0u);
+                    }
                 }
+                if (!ok) break;
                 tc_commit(bar(kODone));
                 if (j + 1 == n) tc_commit(bar(kOFinal));
                 tc_commit(bar(kVEmpty + st));
@@ -381,60 +386,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax warps
+        // Warps w and w+4 hold the same rows; each owns half of every key tile, its
+        // own running max and sum and its own O accumulator, so the two work
+        // independently until the epilogue combines them.
         const int quarter = warp & 3;  // TMEM lanes 32*quarter .. (query rows)
-        const int h = warp >> 2;       // key half of every tile, and half of O's columns
+        const int h = warp >> 2;       // key half of every tile
         const int row = quarter * 32 + lane;
         const int qrow = it.q0 + row;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t tO = tmem + lane_base + kTmemO + h * (D / 2);
+        const uint32_t tO = tmem + lane_base + kTmemO + h * D;
         const int64_t ring_last_r = (p.len > p.S) ? (p.len - 1 - p.S) % p.R : 0;
         const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
-        // Exchange area: [tile parity][half][row] maxima, then ok flags per warp.
-        volatile float* xmax = xchg;
-        volatile int* xok = reinterpret_cast<volatile int*>(xchg + 2 * 2 * 128);
-        volatile float* xsum = xchg + 2 * 2 * 128 + 2 * 2 * 4;
+        volatile float* xm = xchg;        // [half][row] running max
+        volatile float* xl = xchg + 256;  // [half][row] row sum
         float m_run = -INFINITY;
-        float l_run = 0.f;  // this thread's half of the row sum
+        float l_run = 0.f;
         bool ok = true;
-        // Q row -> TMEM (lane = row, bf16 pairs along D): QK then reads only K from
-        // shared memory. Each half copies D/2 elements of its row out of the
-        // 128-byte-swizzled TMA tile (16-byte chunk c of row r sits at c ^ (r % 8)).
-        if (__all_sync(0xffffffffu, mbar_wait(bar(kQFull), 0, abort_flag))) {
-            constexpr int kChunks = D / 16;  // 16-byte chunks per half row
-            uint32_t qv[kChunks * 4];
-#pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-                const int e0 = h * (D / 2) + c * 8;
-                const uint32_t addr = sQ + (e0 / 64) * kTileBytesPerColBlock + row * 128 +
-                                      ((((e0 % 64) / 8) ^ (row & 7)) * 16);
-                const uint4 v4 = lds128(addr);
-                qv[c * 4 + 0] = v4.x;
-                qv[c * 4 + 1] = v4.y;
-                qv[c * 4 + 2] = v4.z;
-                qv[c * 4 + 3] = v4.w;
-            }
-            const uint32_t tq = tmem + lane_base + kTmemQ + h * (D / 4);
-            if constexpr (D == 128) tmem_st32(tq, qv);
-            else tmem_st16(tq, qv);
-            tc_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kQTmem));
-        } else {
-            ok = false;
-            record_abort(p.err, abort_flag);
-        }
         for (int j = 0; j < n; ++j) {
             const int buf = j & 1;
             const uint32_t tS = tmem + lane_base + buf * kTileK;
-            // Waits that guard warp-collective tcgen05 instructions are warp-uniform;
-            // the two warps of a pair also leave the loop together (the named barrier
-            // below has no timeout).
-            const bool ok_s = ok && __all_sync(0xffffffffu, mbar_wait(bar(kSFull + buf), (j >> 1) & 1, abort_flag));
+            // Waits that guard warp-collective tcgen05 instructions are warp-uniform.
+            if (!(ok && __all_sync(0xffffffffu, mbar_wait(bar(kSFull + buf), (j >> 1) & 1, abort_flag)))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
             float s[kHalf];
-            float mh = -INFINITY;
-            if (ok_s) {
-                tc_fence_after();
+            {
                 uint32_t r[2][32];
                 tmem_ld32(tS + h * kHalf, r[0]);
                 tmem_ld32(tS + h * kHalf + 32, r[1]);
@@ -443,41 +421,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[c][i]);
-                int src, row0;
-                tile_of(it, j, src, row0);
-                const bool full =
-                    it.retr && ((src == 0 && row0 + kTileK <= p.len) || (src == 2 && row0 + kTileK <= it.q0));
-                if (!full) {
-#pragma unroll
-                    for (int w = 0; w < 2; ++w) {
-                        const uint32_t bits = visible_bits(p, it.retr, src, row0, 2 * h + w, qrow, ring_last_r);
-#pragma unroll
-                        for (int k = 0; k < 32; ++k)
-                            if (!((bits >> k) & 1u)) s[w * 32 + k] = -INFINITY;
-                    }
-                }
-                float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-                static_assert(kHalf % 8 == 0, "the max loop covers exactly [0, kHalf)");
-#pragma unroll
-                for (int i = 0; i < kHalf; i += 8) {
-                    m0 = fmax3(m0, s[i], s[i + 1]);
-                    m1 = fmax3(m1, s[i + 2], s[i + 3]);
-                    m2 = fmax3(m2, s[i + 4], s[i + 5]);
-                    m3 = fmax3(m3, s[i + 6], s[i + 7]);
-                }
-                mh = fmax3(fmaxf(m0, m1), m2, m3);
             }
-            xmax[(buf * 2 + h) * 128 + row] = mh;
-            if (lane == 0) xok[(buf * 2 + h) * 4 + quarter] = ok_s ? 1 : 0;
-            pair_sync(quarter);
-            const float mo = xmax[(buf * 2 + (1 - h)) * 128 + row];
-            const bool ok_o = xok[(buf * 2 + (1 - h)) * 4 + quarter] != 0;
-            if (!ok_s || !ok_o) {
-                ok = false;
-                break;
+            int src, row0;
+            tile_of(it, j, src, row0);
+            const bool full =
+                it.retr && ((src == 0 && row0 + kTileK <= p.len) || (src == 2 && row0 + kTileK <= it.q0));
+            if (!full) {
+#pragma unroll
+                for (int w = 0; w < 2; ++w) {
+                    const uint32_t bits = visible_bits(p, it.retr, src, row0, 2 * h + w, qrow, ring_last_r);
+#pragma unroll
+                    for (int k = 0; k < 32; ++k)
+                        if (!((bits >> k) & 1u)) s[w * 32 + k] = -INFINITY;
+                }
             }
-            // Both halves of the row see the same max and take the same decision.
-            const float mt = fmaxf(mh, mo) * p.scale_log2;
+            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+            static_assert(kHalf % 8 == 0, "the max loop covers exactly [0, kHalf)");
+#pragma unroll
+            for (int i = 0; i < kHalf; i += 8) {
+                m0 = fmax3(m0, s[i], s[i + 1]);
+                m1 = fmax3(m1, s[i + 2], s[i + 3]);
+                m2 = fmax3(m2, s[i + 4], s[i + 5]);
+                m3 = fmax3(m3, s[i + 6], s[i + 7]);
+            }
+            const float mt = fmax3(fmaxf(m0, m1), m2, m3) * p.scale_log2;
             float factor = 1.f;
             if (mt > m_run + kRescaleThreshold) {  // also taken when m_run is -inf and mt finite
                 factor = fast_exp2(m_run - mt);
@@ -500,15 +467,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2unpack(fadd2(acc2[0], acc2[1]), a0, a1);
             l_run = l_run * factor + (a0 + a1);
             tmem_st32(tS + kTmemP + h * (kHalf / 2), pk);  // P of this half (S columns already read)
-            // O must be complete before it is rescaled: PV(j-1) is the last MMA that
-            // wrote it (kODone completes one phase per PV; the commit behind S(j)
-            // covered PV(j-2)). Each half rescales its own D/2 columns.
+            // O_h must be complete before it is rescaled: PV(j-1) is the last MMA that
+            // wrote it (kODone completes one phase per key tile; the commit behind
+            // S(j) covered PV(j-2)).
             if (j >= 1 && __any_sync(0xffffffffu, factor != 1.f)) {
                 if (__all_sync(0xffffffffu, mbar_wait(bar(kODone), (j - 1) & 1, abort_flag))) {
                     tc_fence_after();
                     uint32_t r[32];
 #pragma unroll
-                    for (int c = 0; c < D / 64; ++c) {
+                    for (int c = 0; c < D / 32; ++c) {
                         tmem_ld32(tO + c * 32, r);
                         tc_wait_ld();
 #pragma unroll
@@ -516,37 +483,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_st32(tO + c * 32, r);
                     }
                 } else {
-                    ok = false;  // the pair leaves together at the next exchange
+                    ok = false;
                     record_abort(p.err, abort_flag);
                 }
             }
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kPFull + buf));
+            if (lane == 0) mbar_arrive(bar((h ? kP1Full : kP0Full) + buf));
+            if (!ok) break;
         }
-        // Row sum of both halves, then the output: each half writes its D/2 columns.
-        xsum[h * 128 + row] = l_run;
+        // Combine the halves: O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)),
+        // each thread of a pair writing D/2 of the row's columns.
+        xm[h * 128 + row] = m_run;
+        xl[h * 128 + row] = l_run;
         pair_sync(quarter);
-        const float l_all = l_run + xsum[(1 - h) * 128 + row];
+        const float m_o = xm[(1 - h) * 128 + row];
+        const float l_o = xl[(1 - h) * 128 + row];
+        const float m_all = fmaxf(m_run, m_o);  // finite: every row sees at least its own key
+        const float f_self = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_all);
+        const float f_o = (m_o == -INFINITY) ? 0.f : fast_exp2(m_o - m_all);
+        const float inv = 1.f / (l_run * f_self + l_o * f_o);
+        const float f0 = (h == 0 ? f_self : f_o) * inv;
+        const float f1 = (h == 0 ? f_o : f_self) * inv;
         if (__all_sync(0xffffffffu, ok && mbar_wait(bar(kOFinal), 0, abort_flag))) {
             tc_fence_after();
-            const float inv = 1.f / l_all;
+            const uint32_t tO0 = tmem + lane_base + kTmemO + h * (D / 2);
             bf16* orow = p.out + ((static_cast<int64_t>(it.b) * p.C + qrow) * p.Hq + it.head) * D + h * (D / 2);
-            uint32_t r[32];
+            uint32_t r0[32], r1[32];
 #pragma unroll
             for (int c = 0; c < D / 64; ++c) {
-                tmem_ld32(tO + c * 32, r);
+                tmem_ld32(tO0 + c * 32, r0);
+                tmem_ld32(tO0 + D + c * 32, r1);
                 tc_wait_ld();
                 if (qrow < p.C) {
 #pragma unroll
                     for (int v8 = 0; v8 < 4; ++v8) {
-                        uint4 o;
-                        o.x = pack_bf16x2(__uint_as_float(r[v8 * 8 + 0]) * inv, __uint_as_float(r[v8 * 8 + 1]) * inv);
-                        o.y = pack_bf16x2(__uint_as_float(r[v8 * 8 + 2]) * inv, __uint_as_float(r[v8 * 8 + 3]) * inv);
-                        o.z = pack_bf16x2(__uint_as_float(r[v8 * 8 + 4]) * inv, __uint_as_float(r[v8 * 8 + 5]) * inv);
-                        o.w = pack_bf16x2(__uint_as_float(r[v8 * 8 + 6]) * inv, __uint_as_float(r[v8 * 8 + 7]) * inv);
-                        *reinterpret_cast<uint4*>(orow + c * 32 + v8 * 8) = o;
+                        uint32_t w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int e = v8 * 8 + 2 * i;
+                            w[i] = pack_bf16x2(__uint_as_float(r0[e]) * f0 + __uint_as_float(r1[e]) * f1,
+                                               __uint_as_float(r0[e + 1]) * f0 + __uint_as_float(r1[e + 1]) * f1);
+                        }
+                        *reinterpret_cast<uint4*>(orow + c * 32 + v8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
             }
