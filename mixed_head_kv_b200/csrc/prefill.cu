@@ -174,16 +174,49 @@ __device__ __forceinline__ uint32_t bits_below(int64_t x) {
     return (1u << static_cast<uint32_t>(x)) - 1u;
 }
 
+// Bits k of a 32-bit word set for base + k in [lo, hi).
+__device__ __forceinline__ uint32_t bits_in(int64_t lo, int64_t hi, int64_t base) {
+    return bits_below(hi - base) & ~bits_below(lo - base);
+}
+
+// Ring slots of the streaming cache visible from one query row, as at most two
+// slot ranges [a0, b0) and [a1, b1). The ring holds the latest min(recent,
+// len - sink) positions p >= sink below len, position p in slot
+// sink + (p - sink) mod recent; the query at len + qrow sees those with
+// p > len + qrow - recent, a contiguous run of positions [lo, len) that wraps
+// at most once in slot order.
+struct RingVis {
+    int64_t a0, b0, a1, b1;
+};
+
+__device__ __forceinline__ RingVis ring_visible(const PrefillParams& p, int qrow) {
+    RingVis g{0, 0, 0, 0};
+    int64_t lo = p.len + qrow - p.R + 1;
+    if (lo < p.S) lo = p.S;
+    const int64_t c = p.len - lo;
+    if (c > 0) {
+        const int64_t r0 = (lo - p.S) % p.R;
+        g.a0 = p.S + r0;
+        if (r0 + c <= p.R) {
+            g.b0 = p.S + r0 + c;
+        } else {
+            g.b0 = p.S + p.R;
+            g.a1 = p.S;
+            g.b1 = p.S + r0 + c - p.R;
+        }
+    }
+    return g;
+}
+
 // Visibility of keys [32w, 32w+32) of tile (src, row0) from chunk query row
 // `qrow` (absolute position len + qrow), one bit per key.
 //   src 0 (retrieval cache): slot j holds position j, valid for j < len.
-//   src 1 (streaming cache): sink slots j < sink hold position j; ring slot
-//     sink + r holds the latest position p < len with (p - sink) mod recent == r;
-//     visible when inside the query's window.
+//   src 1 (streaming cache): sink slots j < sink hold position j, valid for
+//     j < len; ring slots as in ring_visible.
 //   src 2 (chunk): row c is position len + c, valid for c < C, causal, and for
 //     streaming heads a sink (len + c < sink) or inside the window.
 __device__ __forceinline__ uint32_t visible_bits(const PrefillParams& p, int retr, int src, int row0, int w,
-                                                 int qrow, int64_t ring_last_r) {
+                                                 int qrow, const RingVis& ring) {
     const int64_t L = p.len;
     const int base = row0 + 32 * w;
     if (src == 0) return bits_below(L - base);
@@ -195,25 +228,8 @@ __device__ __forceinline__ uint32_t visible_bits(const PrefillParams& p, int ret
         const uint32_t band = ~bits_below(static_cast<int64_t>(qrow) - p.R + 1 - base);
         return causal & (sink | band);
     }
-    const int64_t pq = L + qrow;
-    const int64_t last = L - 1;
-    uint32_t bits = 0;
-    for (int k = 0; k < 32; ++k) {
-        const int64_t slot = base + k;
-        bool vis;
-        if (slot < p.S) {
-            vis = slot < L;
-        } else if (slot < p.W && L > p.S) {
-            const int64_t r = slot - p.S;
-            const int64_t back = (r <= ring_last_r) ? (ring_last_r - r) : (ring_last_r - r + p.R);
-            const int64_t pos = last - back;
-            vis = (pos >= p.S) && (pq - pos < p.R);
-        } else {
-            vis = false;
-        }
-        bits |= static_cast<uint32_t>(vis) << k;
-    }
-    return bits;
+    const int64_t sink_hi = L < p.S ? L : p.S;
+    return bits_in(0, sink_hi, base) | bits_in(ring.a0, ring.b0, base) | bits_in(ring.a1, ring.b1, base);
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -395,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qrow = it.q0 + row;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t tO = tmem + lane_base + kTmemO + h * D;
-        const int64_t ring_last_r = (p.len > p.S) ? (p.len - 1 - p.S) % p.R : 0;
+        const RingVis ring = ring_visible(p, qrow);
         const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
         volatile float* xm = xchg;        // [half][row] running max
         volatile float* xl = xchg + 256;  // [half][row] row sum
@@ -429,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!full) {
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
-                    const uint32_t bits = visible_bits(p, it.retr, src, row0, 2 * h + w, qrow, ring_last_r);
+                    const uint32_t bits = visible_bits(p, it.retr, src, row0, 2 * h + w, qrow, ring);
 #pragma unroll
                     for (int k = 0; k < 32; ++k)
                         if (!((bits >> k) & 1u)) s[w * 32 + k] = -INFINITY;
