@@ -616,6 +616,42 @@ def run_sweep(args):
     return out
 
 
+# ----------------------------------------------------------------------------- memory footprint
+# Model shapes for the footprint table: (name, layers, q heads, KV heads, head_dim, retrieval ratio,
+# parameters). The parameter counts are the public sizes of the models these shapes follow; they
+# only add the bf16 weights to both sides of the whole-model ratio.
+FOOTPRINT_MODELS = (
+    ("llama2_7b_mha", 32, 32, 32, 128, 0.25, 6.74e9),
+    ("llama3_8b_gqa", 32, 32, 8, 128, 0.5, 8.03e9),
+)
+
+
+def memory_footprint(duo, name, layers, hq, hkv, d, ratio, params, context, sink=64, recent=256, batch=1):
+    """KV-cache bytes of full attention against the mixed-head cache the library sizes
+    (duo_cache_alloc without a buffer), for one batch at `context` tokens."""
+    w = workloads.Workload(name, batch=batch, num_q_heads=hq, num_kv_heads=hkv, head_dim=d, sink=sink,
+                           recent=recent, retrieval_ratio=ratio, num_layers=layers)
+    mask = [m for l in range(layers) for m in workloads.retrieval_mask(w, l)]
+    lay = duo.make_layout(layers, batch, hq, hkv, d, sink, recent, context)
+    st, required, _ = duo.duo_cache_alloc(lay, mask)
+    if st != duo.DUO_OK:
+        raise RuntimeError(duo.duo_status_str(st))
+    n_retr = sum(mask)
+    kv_full = layers * batch * hkv * context * d * 2 * 2
+    kv_duo = (n_retr * context + (len(mask) - n_retr) * (sink + recent)) * batch * d * 2 * 2
+    weights = params * 2
+    return {"model": name, "context": context, "batch": batch, "retrieval_kv_heads": n_retr,
+            "kv_full_bytes": kv_full, "kv_duo_bytes": kv_duo, "duo_required_bytes": required,
+            "kv_ratio": kv_full / kv_duo, "with_weights_ratio": (weights + kv_full) / (weights + required)}
+
+
+def run_memory(args):
+    import mixed_head_kv_b200 as duo
+    for m in FOOTPRINT_MODELS:
+        for context in (32768, 131072, 1 << 20):
+            print(json.dumps(memory_footprint(duo, *m, context)), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -625,7 +661,12 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--sweep", action="store_true",
                     help="time the other workloads (GQA decode at 128K and 1M, MHA ratio sweep) instead")
+    ap.add_argument("--memory", action="store_true",
+                    help="print the KV-cache footprint of full attention against the mixed-head cache (no GPU)")
     args = ap.parse_args(argv)
+    if args.memory:
+        run_memory(args)
+        return
     if args.sweep:
         run_sweep(args)
         return
