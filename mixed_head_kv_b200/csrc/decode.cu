@@ -29,22 +29,25 @@ namespace duo {
 namespace {
 
 constexpr int kWarps = kDecodeThreads / 32;
-constexpr int kStages = 3;
 constexpr int kGroupRows = 4;  // row groups accumulated per register batch
 // Rows per warp hinted into L2 before the wait for the previous kernel (32 KB of
 // K and V at D = 128).
 template <int D>
 constexpr int64_t kPrefetchRows = 16384 / (D * 2);
 
-template <int D>
+// Ring depth and residency per group size: for G = 2 and 4 (issue-heavy rows)
+// three CTAs of 2-stage rings per SM hide latency better than two of 3 stages;
+// the same bytes are in flight either way.
+template <int D, int G>
 struct Geom {
+    static constexpr int kStages = (G == 2 || G == 4) ? 2 : 3;
     static constexpr int LPR = D / 8;                 // lanes per row
     static constexpr int RPW = 32 / LPR;              // rows per warp instruction
     static constexpr int BLK = 4096 / (D * 2);        // rows per 4 KB block
     static constexpr int kBlockBytes = BLK * D * 2;   // one K (or V) block
     static constexpr int kStageBytes = 2 * kBlockBytes;
     static constexpr int kWarpBytes = kStages * kStageBytes;
-    static constexpr int kRingBytes = kWarps * kWarpBytes;  // 96 KB
+    static constexpr int kRingBytes = kWarps * kWarpBytes;  // 96 KB (3 stages) or 64 KB
     static constexpr int kBarOff = kRingBytes;
     static constexpr int kSmem = kBarOff + kWarps * kStages * 8 + 16;
 };
@@ -173,13 +176,13 @@ __device__ __forceinline__ void merge_lanes(DecState<G>& st, int off) {
 template <int D, int G>
 __device__ bool warp_stream(DecState<G>& st, const uint64_t (&q2)[G][4], const bf16* kbase, const bf16* vbase,
                             int64_t r0, int64_t r1, int64_t skip, uint32_t ring, uint32_t bars) {
-    using Gm = Geom<D>;
+    using Gm = Geom<D, G>;
     const int lane = threadIdx.x & 31;
     const int sub = lane % Gm::LPR;
     const int rsub = lane / Gm::LPR;
     const int64_t nblk = (r1 - r0 + Gm::BLK - 1) / Gm::BLK;
     auto issue = [&](int64_t i) {
-        const int stg = static_cast<int>(i % kStages);
+        const int stg = static_cast<int>(i % Gm::kStages);
         const int64_t a = r0 + i * Gm::BLK;
         const int64_t n = (r1 - a < Gm::BLK) ? (r1 - a) : Gm::BLK;
         const uint32_t bytes = static_cast<uint32_t>(n * D * 2);
@@ -190,15 +193,15 @@ __device__ bool warp_stream(DecState<G>& st, const uint64_t (&q2)[G][4], const b
         bulk_load(dst + Gm::kBlockBytes, vbase + a * D, bytes, bar);
     };
     if (lane == 0) {
-        for (int64_t i = 0; i < nblk && i < kStages; ++i) issue(i);
+        for (int64_t i = 0; i < nblk && i < Gm::kStages; ++i) issue(i);
     }
     for (int64_t i = 0; i < nblk; ++i) {
-        const int stg = static_cast<int>(i % kStages);
-        if (!mbar_wait(bars + 8u * stg, static_cast<uint32_t>((i / kStages) & 1), nullptr)) {
+        const int stg = static_cast<int>(i % Gm::kStages);
+        if (!mbar_wait(bars + 8u * stg, static_cast<uint32_t>((i / Gm::kStages) & 1), nullptr)) {
             // Give the copies still in flight one more bounded wait before the
             // CTA moves on (and later reuses this shared memory).
-            for (int64_t j = i + 1; j < nblk && j < i + kStages; ++j)
-                mbar_wait(bars + 8u * static_cast<uint32_t>(j % kStages), static_cast<uint32_t>((j / kStages) & 1),
+            for (int64_t j = i + 1; j < nblk && j < i + Gm::kStages; ++j)
+                mbar_wait(bars + 8u * static_cast<uint32_t>(j % Gm::kStages), static_cast<uint32_t>((j / Gm::kStages) & 1),
                           nullptr);
             return false;
         }
@@ -221,33 +224,33 @@ __device__ bool warp_stream(DecState<G>& st, const uint64_t (&q2)[G][4], const b
             accumulate<D, G, kGroupRows>(st, q2, kx, vx, valid);
         }
         __syncwarp();
-        if (lane == 0 && i + kStages < nblk) {
+        if (lane == 0 && i + Gm::kStages < nblk) {
             fence_proxy_async_smem();  // our generic reads of this stage precede the async refill
-            issue(i + kStages);
+            issue(i + Gm::kStages);
         }
     }
     return true;
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams p) {
-    using Gm = Geom<D>;
+__device__ __forceinline__ void decode_body(const DecodeParams& p) {
+    using Gm = Geom<D, G>;
     constexpr int LPR = Gm::LPR;
     extern __shared__ __align__(128) uint8_t smem[];
     // After the streaming phase the ring is reused for the cross-warp merge.
     float* sm_m = reinterpret_cast<float*>(smem);                 // [kWarps][G]
     float* sm_l = sm_m + kWarps * G;                              // [kWarps][G]
     float* sm_o = sm_l + kWarps * G;                              // [kWarps][G][D]
-    int* sm_last = reinterpret_cast<int*>(smem + Gm::kBarOff + kWarps * kStages * 8);
+    int* sm_last = reinterpret_cast<int*>(smem + Gm::kBarOff + kWarps * Gm::kStages * 8);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const int sub = lane % LPR;
     const uint32_t ring = smem_u32(smem) + warp * Gm::kWarpBytes;
-    const uint32_t bars = smem_u32(smem) + Gm::kBarOff + warp * kStages * 8;
+    const uint32_t bars = smem_u32(smem) + Gm::kBarOff + warp * Gm::kStages * 8;
     if (lane == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(bars + 8u * s, 1);
+        for (int s = 0; s < Gm::kStages; ++s) mbar_init(bars + 8u * s, 1);
         fence_barrier_init();
     }
     __syncwarp();
@@ -478,16 +481,34 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
     if (tid == 0) p.counters[b * p.Hkv + g] = 0u;  // ready for the next step (stream-ordered)
 }
 
+// The kernel, with the register budget its residency needs: three CTAs per SM
+// for G = 2 and 4, the compiler's own choice otherwise.
+template <int D, int G>
+__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams p) {
+    decode_body<D, G>(p);
+}
+template <int D, int G>
+__global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel_3(const DecodeParams p) {
+    decode_body<D, G>(p);
+}
+
 template <int D, int G>
 cudaError_t launch_dg(const DecodeParams& p, unsigned grid, cudaStream_t s) {
-    constexpr int smem = Geom<D>::kSmem;
-    static_assert((kWarps * 2 * G + kWarps * G * D) * 4 <= Geom<D>::kRingBytes, "warp merge arrays fit in the ring");
-    static_assert((16 + 8) * (G * D / 4 >= kDecodeThreads ? G * D / 4 : kDecodeThreads) <= Geom<D>::kRingBytes,
+    constexpr int smem = Geom<D, G>::kSmem;
+    static_assert((kWarps * 2 * G + kWarps * G * D) * 4 <= Geom<D, G>::kRingBytes, "warp merge arrays fit in the ring");
+    static_assert((16 + 8) * (G * D / 4 >= kDecodeThreads ? G * D / 4 : kDecodeThreads) <= Geom<D, G>::kRingBytes,
                   "split merge arrays fit in the ring");
     static SmemLimitOnce limit;
-    cudaError_t e = limit.apply(reinterpret_cast<const void*>(&decode_kernel<D, G>), smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(decode_kernel<D, G>, dim3(grid), dim3(kDecodeThreads), smem, s, p);
+    static_assert(decode_ctas_per_sm(G) == 2 || decode_ctas_per_sm(G) == 3, "one of the two kernels");
+    if constexpr (decode_ctas_per_sm(G) == 3) {
+        const cudaError_t e = limit.apply(reinterpret_cast<const void*>(&decode_kernel_3<D, G>), smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(decode_kernel_3<D, G>, dim3(grid), dim3(kDecodeThreads), smem, s, p);
+    } else {
+        const cudaError_t e = limit.apply(reinterpret_cast<const void*>(&decode_kernel<D, G>), smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(decode_kernel<D, G>, dim3(grid), dim3(kDecodeThreads), smem, s, p);
+    }
 }
 
 template <int D>

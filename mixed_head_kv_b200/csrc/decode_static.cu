@@ -99,7 +99,8 @@ extern "C" duo_status duo_decode_static_scratch(duo_cache* c, int32_t layer, con
 
     // Same split plan as duo_decode, then limited to what the array holds.
     const int64_t rows = p.len + 1;
-    int64_t nsplit = plan_decode_splits(L.batch, p.n_retr, p.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms);
+    int64_t nsplit =
+        plan_decode_splits(L.batch, p.n_retr, p.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms, c->G);
     const size_t counters_bytes = round256(static_cast<size_t>(L.batch) * L.num_kv_heads * sizeof(uint32_t));
     if (p.n_retr > 0) {
         const int64_t pairs = static_cast<int64_t>(L.batch) * p.n_retr;

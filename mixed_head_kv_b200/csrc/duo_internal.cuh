@@ -80,7 +80,9 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 constexpr int kDecodeMaxSplits = 256;
 constexpr int kDecodeThreads = 128;
 
-constexpr int kDecodeCtasPerSm = 2;  // residency of decode_kernel (96 KB of shared memory each)
+// Resident decode CTAs per SM for a query-group size (the kernel's shared memory
+// and register budget are sized for it).
+__host__ __device__ constexpr int decode_ctas_per_sm(int G) { return (G == 2 || G == 4) ? 3 : 2; }
 
 // Splits per retrieval (b, KV head) for one decode step. Every CTA streams
 // its rows at about the same rate, so the step takes about
@@ -89,12 +91,12 @@ constexpr int kDecodeCtasPerSm = 2;  // residency of decode_kernel (96 KB of sha
 // sink + recent rows each. Pick the split count (>= 256 rows per split, at most
 // kDecodeMaxSplits) that minimises that estimate.
 inline int64_t plan_decode_splits(int64_t batch, int64_t n_retr, int64_t n_strm, int64_t rows, int64_t strm_rows,
-                                  int num_sms) {
+                                  int num_sms, int G) {
     if (n_retr <= 0) return 1;
     constexpr int64_t kCtaCostRows = 64;
     const int64_t pairs = batch * n_retr;
     const int64_t strm_items = batch * n_strm;
-    const int64_t slots = static_cast<int64_t>(num_sms) * kDecodeCtasPerSm;
+    const int64_t slots = static_cast<int64_t>(num_sms) * decode_ctas_per_sm(G);
     int64_t max_split = (rows + 255) / 256;
     if (max_split > kDecodeMaxSplits) max_split = kDecodeMaxSplits;
     if (max_split < 1) max_split = 1;
@@ -197,7 +199,8 @@ inline int64_t decode_plan(duo_cache* c, int32_t layer, int64_t rows) {
     if (c->plan_key[layer] != key) {
         const duo::DecodeParams& t = c->decode_tmpl[layer];
         c->plan_nsplit[layer] =
-            duo::plan_decode_splits(c->lay.batch, t.n_retr, t.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms);
+            duo::plan_decode_splits(c->lay.batch, t.n_retr, t.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms,
+                                    c->G);
         c->plan_key[layer] = key;
     }
     return c->plan_nsplit[layer];
