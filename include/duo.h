@@ -61,9 +61,15 @@ typedef enum duo_status {
 #define DUO_MAX_Q_HEADS 256
 #define DUO_MAX_KV_HEADS 128
 
+/* Largest batch whose sequences may have different lengths (a ragged batch):
+ * the per-sequence lengths travel with each launch. Larger batches keep one
+ * length for all sequences. */
+#define DUO_MAX_RAGGED_BATCH 64
+
 /* Shape of the model's attention and of the caches.
  *   num_layers    >= 1
- *   batch         >= 1 sequences, all of the same length
+ *   batch         >= 1 sequences (each with its own cache length; see
+ *                 duo_cache_seq_lens)
  *   num_q_heads   query heads, a multiple of num_kv_heads (GQA group size G)
  *   num_kv_heads  KV heads; the retrieval/streaming type is per (layer, KV head)
  *   head_dim      64 or 128
@@ -119,14 +125,27 @@ DUO_API duo_status duo_cache_free(duo_cache* cache);
  * (the per-head cache update of DuoAttention: retrieval heads keep everything,
  * streaming heads keep sinks and evict the oldest recent token).
  *   k, v   device [batch][n_tok][num_kv_heads][head_dim] bf16, the tokens at
- *          positions [len, len + n_tok) with len = duo_cache_len(layer)
+ *          positions [len_b, len_b + n_tok) of each sequence b (its own length)
  *   n_tok  >= 0 (0 is a no-op)
  * Retrieval heads write position p to slot p. Streaming heads write sink
  * positions to their slots and only the last min(n_tok, recent) non-sink
  * positions to their ring slots (earlier ones would be evicted within the call).
- * DUO_ERR_CAPACITY if len + n_tok > max_len. Then len += n_tok. */
+ * DUO_ERR_CAPACITY if some len_b + n_tok > max_len. Then every len_b += n_tok. */
 DUO_API duo_status duo_cache_append(duo_cache* cache, int32_t layer, const void* k, const void* v, int64_t n_tok,
                             void* stream);
+
+/* duo_cache_append_ragged — append a different number of tokens to each
+ * sequence of `layer` (a ragged batch: sequences of different lengths).
+ *   k, v     device [batch][max_tok][num_kv_heads][head_dim]; sequence b's rows
+ *            [0, n_tok[b]) are its tokens at positions [len_b, len_b + n_tok[b]),
+ *            the remaining rows are not read
+ *   n_tok    host [batch], 0 <= n_tok[b] <= max_tok
+ * Same slot rules as duo_cache_append, per sequence. Needs batch <=
+ * DUO_MAX_RAGGED_BATCH unless every sequence has the same length and
+ * n_tok[b] == max_tok for all b. DUO_ERR_CAPACITY if some len_b + n_tok[b] >
+ * max_len (nothing is appended). Then len_b += n_tok[b]. */
+DUO_API duo_status duo_cache_append_ragged(duo_cache* cache, int32_t layer, const void* k, const void* v,
+                                   const int64_t* n_tok, int64_t max_tok, void* stream);
 
 /* duo_prefill — attention of one prefill chunk of `layer` (DuoAttention
  * pre-filling; chunked as in the chunked-prefill work the pages cite).
@@ -138,29 +157,43 @@ DUO_API duo_status duo_cache_append(duo_cache* cache, int32_t layer, const void*
  * streaming heads over the sinks and the recent window, read from the
  * streaming cache for positions < len and from k/v for the chunk.
  * Does NOT modify the cache: call duo_cache_append(layer, k, v, n_tok) after it.
+ * All sequences must have the same length (DUO_ERR_STATE otherwise).
  * DUO_ERR_CAPACITY if a retrieval head could not hold len + n_tok tokens. */
 DUO_API duo_status duo_prefill(duo_cache* cache, int32_t layer, const void* q, const void* k, const void* v, void* out,
                        int64_t n_tok, void* stream);
 
 /* duo_decode — one decoding step of `layer` (DuoAttention decoding).
- *   q            device [batch][num_q_heads][head_dim], queries at position len
- *   k_new, v_new device [batch][num_kv_heads][head_dim], the new token
+ *   q            device [batch][num_q_heads][head_dim], sequence b's query at
+ *                position len_b (its cache length)
+ *   k_new, v_new device [batch][num_kv_heads][head_dim], the new tokens
  *   out          device [batch][num_q_heads][head_dim], written
- * Appends the new token to every head's cache (as duo_cache_append with one
- * token), then attends: retrieval heads over positions [0, len], streaming
- * heads over the sinks and the last `recent` positions. Then len += 1.
+ * Appends each sequence's new token to every head's cache at that sequence's
+ * own length (as duo_cache_append with one token), then attends: retrieval
+ * heads over positions [0, len_b], streaming heads over the sinks and the last
+ * `recent` positions. Then every len_b += 1. Sequences of different lengths
+ * (a ragged batch) need batch <= DUO_MAX_RAGGED_BATCH, else DUO_ERR_STATE.
  * Uses the cache's decode scratch: decode calls on one cache must not overlap
- * on the device. DUO_ERR_CAPACITY if len + 1 > max_len. */
+ * on the device. DUO_ERR_CAPACITY if some len_b + 1 > max_len. */
 DUO_API duo_status duo_decode(duo_cache* cache, int32_t layer, const void* q, const void* k_new, const void* v_new,
                       void* out, void* stream);
 
-/* duo_cache_len — tokens appended so far to `layer` (host value; no sync). */
+/* duo_cache_len — tokens appended so far to `layer` (host value; no sync).
+ * DUO_ERR_STATE if its sequences have different lengths (see
+ * duo_cache_seq_lens). */
 DUO_API duo_status duo_cache_len(const duo_cache* cache, int32_t layer, int64_t* len);
 
-/* duo_cache_set_len — set the host-side length of `layer`, e.g. to restore a
- * snapshot taken with duo_cache_len (the device contents are the caller's to
- * restore). 0 <= len <= max_len. */
+/* duo_cache_set_len — set the host-side length of every sequence of `layer`,
+ * e.g. to restore a snapshot taken with duo_cache_len (the device contents are
+ * the caller's to restore). 0 <= len <= max_len. */
 DUO_API duo_status duo_cache_set_len(duo_cache* cache, int32_t layer, int64_t len);
+
+/* duo_cache_seq_lens — per-sequence lengths of `layer`.
+ *   lens  host [batch], written (host values; no sync) */
+DUO_API duo_status duo_cache_seq_lens(const duo_cache* cache, int32_t layer, int64_t* lens);
+
+/* duo_cache_set_seq_lens — set the per-sequence lengths of `layer`.
+ *   lens  host [batch], 0 <= lens[b] <= max_len (nothing changes otherwise) */
+DUO_API duo_status duo_cache_set_seq_lens(duo_cache* cache, int32_t layer, const int64_t* lens);
 
 /* duo_cache_views — where one KV head's cache lives, for inspection.
  *   k, v          out: device pointers to [batch][slots][head_dim] bf16

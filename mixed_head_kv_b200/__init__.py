@@ -37,9 +37,12 @@ DUO_STATIC_SCRATCH_BYTES = 16 * 1024 * 1024
 DUO_MAX_Q_HEADS = 256
 DUO_MAX_KV_HEADS = 128
 
+DUO_MAX_RAGGED_BATCH = 64  # sequences of different lengths per batch (include/duo.h)
+
 EXPORTED = ("duo_cache_alloc", "duo_cache_free", "duo_cache_append", "duo_prefill", "duo_decode",
             "duo_cache_len", "duo_cache_set_len", "duo_cache_views", "duo_cache_error", "duo_status_str",
-            "duo_decode_static_scratch")
+            "duo_decode_static_scratch", "duo_cache_append_ragged", "duo_cache_seq_lens",
+            "duo_cache_set_seq_lens")
 
 
 class duo_layout(ctypes.Structure):
@@ -76,6 +79,12 @@ _lib.duo_cache_set_len.argtypes = [_P, _I32, _I64]
 _lib.duo_cache_views.restype = _ST
 _lib.duo_cache_views.argtypes = [_P, _I32, _I32, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_I64),
                                  ctypes.POINTER(_I32)]
+_lib.duo_cache_append_ragged.restype = _ST
+_lib.duo_cache_append_ragged.argtypes = [_P, _I32, _P, _P, ctypes.POINTER(_I64), _I64, _P]
+_lib.duo_cache_seq_lens.restype = _ST
+_lib.duo_cache_seq_lens.argtypes = [_P, _I32, ctypes.POINTER(_I64)]
+_lib.duo_cache_set_seq_lens.restype = _ST
+_lib.duo_cache_set_seq_lens.argtypes = [_P, _I32, ctypes.POINTER(_I64)]
 _lib.duo_cache_error.restype = _ST
 _lib.duo_cache_error.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
 
@@ -170,6 +179,24 @@ def duo_cache_set_len(handle, layer, length) -> int:
     return _lib.duo_cache_set_len(handle, layer, length)
 
 
+def duo_cache_append_ragged(handle, layer, k, v, n_tok: Sequence[int], max_tok: int, stream=None) -> int:
+    """Sequence b appends rows [0, n_tok[b]) of k/v [batch][max_tok][Hkv][D]."""
+    n = (_I64 * max(1, len(n_tok)))(*[int(x) for x in n_tok])
+    return _lib.duo_cache_append_ragged(handle, layer, _ptr(k), _ptr(v), n, max_tok,
+                                        _stream(stream) if k is not None else None)
+
+
+def duo_cache_seq_lens(handle, layer, batch: int):
+    lens = (_I64 * batch)()
+    st = _lib.duo_cache_seq_lens(handle, layer, lens)
+    return st, list(lens)
+
+
+def duo_cache_set_seq_lens(handle, layer, lens: Sequence[int]) -> int:
+    arr = (_I64 * max(1, len(lens)))(*[int(x) for x in lens])
+    return _lib.duo_cache_set_seq_lens(handle, layer, arr)
+
+
 def duo_cache_views(handle, layer, kv_head):
     k, v, slots, r = _P(), _P(), _I64(0), _I32(0)
     st = _lib.duo_cache_views(handle, layer, kv_head, ctypes.byref(k), ctypes.byref(v), ctypes.byref(slots),
@@ -215,6 +242,19 @@ class DuoCache:
 
     def append(self, layer, k, v, stream=None):
         _check(duo_cache_append(self.handle, layer, k, v, k.shape[1], stream), "duo_cache_append")
+
+    def append_ragged(self, layer, k, v, n_tok, stream=None):
+        """Per-sequence token counts n_tok[b] <= k.shape[1] (rows past them are not read)."""
+        _check(duo_cache_append_ragged(self.handle, layer, k, v, n_tok, k.shape[1], stream),
+               "duo_cache_append_ragged")
+
+    def seq_lens(self, layer):
+        st, lens = duo_cache_seq_lens(self.handle, layer, self.layout.batch)
+        _check(st, "duo_cache_seq_lens")
+        return lens
+
+    def set_seq_lens(self, layer, lens):
+        _check(duo_cache_set_seq_lens(self.handle, layer, lens), "duo_cache_set_seq_lens")
 
     def prefill(self, layer, q, k, v, out, stream=None):
         _check(duo_prefill(self.handle, layer, q, k, v, out, q.shape[1], stream), "duo_prefill")

@@ -18,7 +18,6 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
     grid_launch_dependents();
     const int vec_per_row = p.D / 8;
     const int64_t total = static_cast<int64_t>(p.B) * p.n * p.Hkv * vec_per_row;
-    const int64_t first_kept = p.len + p.n - p.R;  // ring positions below this are overwritten in-call
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int e = static_cast<int>(i % vec_per_row);
@@ -27,7 +26,12 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
         r /= p.Hkv;
         const int64_t c = r % p.n;
         const int b = static_cast<int>(r / p.n);
-        const int64_t pos = p.len + c;
+        // Sequence b appends rows [0, n_b) at its own length (ragged batches).
+        const int64_t len_b = p.ragged ? p.seq_len[b] : p.len;
+        const int64_t n_b = p.ragged ? p.seq_n[b] : p.n;
+        if (c >= n_b) continue;
+        const int64_t pos = len_b + c;
+        const int64_t first_kept = len_b + n_b - p.R;  // ring positions below this are overwritten in-call
         const int pool = p.heads.pool_idx[g];
         bf16* dk;
         bf16* dv;
@@ -60,9 +64,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
     const int64_t total = static_cast<int64_t>(p.B) * p.n * p.Hkv * (p.D / 8);
     if (total == 0) return cudaSuccess;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = p.num_sms > 0 ? p.num_sms : 148;
     const int threads = 256;
     int64_t blocks = (total + threads - 1) / threads;
     const int64_t cap = static_cast<int64_t>(sms) * 8;  // grid-stride beyond 8 resident CTAs per SM

@@ -270,7 +270,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
         g = p.strm_list[si % p.n_strm];
     }
     const int pool = p.heads.pool_idx[g];
-    const int64_t L = p.len;  // new token position
+    const int64_t L = p.ragged ? p.seq_len[b] : p.len;  // this sequence's new token position
 
     // Rows of this item held in the cache, and whether it owns the new token.
     const bf16* kbase;
@@ -285,8 +285,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
         vbase = p.pools.rv + head_off;
         r0 = split * p.split_rows;
         const int64_t s1 = r0 + p.split_rows;
-        owns_new = s1 >= L + 1;
-        r1 = owns_new ? L : s1;
+        // Splits are cut for the longest sequence: in a ragged batch a shorter
+        // sequence's last splits hold no rows (they still report to the merge).
+        owns_new = r0 <= L && s1 >= L + 1;
+        r1 = owns_new ? L : (s1 < L ? s1 : (L > r0 ? L : r0));
         new_k_dst = p.pools.rk + head_off + L * D;
         new_v_dst = p.pools.rv + head_off + L * D;
     } else {
@@ -385,18 +387,19 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm_m[w * G + h]);
+        const float Ms = (M == -INFINITY) ? 0.f : M;  // -inf: a split without rows
         float Lsum = 0.f, O = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-            const float f = fast_exp2(sm_m[w * G + h] - M);
+            const float f = fast_exp2(sm_m[w * G + h] - Ms);
             Lsum += f * sm_l[w * G + h];
             O += f * sm_o[(w * G + h) * D + d];
         }
         if (final_now) {
             p.out[(static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d] = __float2bfloat16_rn(O / Lsum);
         } else {
-            p.part_o[(item * G + h) * D + d] = O / Lsum;
-            if (d == 0) p.part_lse[item * G + h] = M + __log2f(Lsum);
+            p.part_o[(item * G + h) * D + d] = Lsum > 0.f ? O / Lsum : 0.f;
+            if (d == 0) p.part_lse[item * G + h] = Lsum > 0.f ? M + __log2f(Lsum) : -INFINITY;
         }
     }
     if (final_now) return;
@@ -434,7 +437,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
         for (int s = rep; s < ns; s += kRep) {
             const float x = __ldcg(pl + static_cast<int64_t>(s) * G + h);
             const float4 o = __ldcg(po + static_cast<int64_t>(s) * kUnits + u);
-            if (x > M) {  // every partial has a finite log-sum-exp
+            if (x > M) {
                 const float f = fast_exp2(M - x);  // 0 while M is -inf
                 Ls *= f;
                 acc.x *= f;
@@ -443,7 +446,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
                 acc.w *= f;
                 M = x;
             }
-            const float w = fast_exp2(x - M);
+            // A split without rows (ragged batch) has lse = -inf and weight 0; a select,
+            // not a branch, keeps the loads of the unrolled iterations together.
+            const float w = (x == -INFINITY) ? 0.f : fast_exp2(x - M);
             Ls += w;
             acc.x = fmaf(w, o.x, acc.x);
             acc.y = fmaf(w, o.y, acc.y);

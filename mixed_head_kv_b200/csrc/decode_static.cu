@@ -67,7 +67,6 @@ extern "C" duo_status duo_decode_static_scratch(duo_cache* c, int32_t layer, con
     if (dev != c->device) return DUO_ERR_STATE;
     if (!q || !k_new || !v_new || !out) return DUO_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return DUO_ERR_ALIGNMENT;
-    if (c->len[layer] + 1 > c->lay.max_len) return DUO_ERR_CAPACITY;
     const duo_layout& L = c->lay;
 
     DecodeParams p{};
@@ -77,7 +76,8 @@ extern "C" duo_status duo_decode_static_scratch(duo_cache* c, int32_t layer, con
     p.out = static_cast<bf16*>(out);
     p.pools = c->pools;
     p.err = c->err;
-    p.len = c->len[layer];
+    if (fill_decode_lengths(c, layer, p) != DUO_OK) return DUO_ERR_STATE;
+    if (p.len + 1 > c->lay.max_len) return DUO_ERR_CAPACITY;
     p.max_len = L.max_len;
     p.B = L.batch;
     p.Hq = L.num_q_heads;
@@ -127,6 +127,7 @@ extern "C" duo_status duo_decode_static_scratch(duo_cache* c, int32_t layer, con
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(p.counters, 0, counters_bytes, s) != cudaSuccess) return DUO_ERR_CUDA;
     if (launch_decode(p, s) != cudaSuccess) return DUO_ERR_CUDA;
-    c->len[layer] += 1;
+    int64_t* lens = seq_lens(c, layer);
+    for (int32_t b = 0; b < L.batch; ++b) lens[b] += 1;
     return DUO_OK;
 }

@@ -177,7 +177,7 @@ duo_status duo_cache_alloc(const duo_layout* layout, const uint8_t* is_retrieval
     for (int64_t i = 0; i < n; ++i) c->pool_idx[i] = is_retrieval[i] ? nr++ : ns++;
     c->n_retr_all = nr;
     c->n_strm_all = ns;
-    c->len.assign(L.num_layers, 0);
+    c->len.assign(static_cast<size_t>(L.num_layers) * L.batch, 0);
     if (cudaGetDevice(&c->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
         delete c;
@@ -250,14 +250,34 @@ duo_status duo_cache_free(duo_cache* cache) {
 
 duo_status duo_cache_len(const duo_cache* c, int32_t layer, int64_t* len) {
     if (!c || !len || layer < 0 || layer >= c->lay.num_layers) return DUO_ERR_INVALID_ARG;
-    *len = c->len[layer];
+    bool uniform = true;
+    const int64_t mx = longest_seq(c, layer, &uniform);
+    if (!uniform) return DUO_ERR_STATE;
+    *len = mx;
     return DUO_OK;
 }
 
 duo_status duo_cache_set_len(duo_cache* c, int32_t layer, int64_t len) {
     if (!c || layer < 0 || layer >= c->lay.num_layers) return DUO_ERR_INVALID_ARG;
     if (len < 0 || len > c->lay.max_len) return DUO_ERR_INVALID_ARG;
-    c->len[layer] = len;
+    int64_t* L = seq_lens(c, layer);
+    for (int32_t b = 0; b < c->lay.batch; ++b) L[b] = len;
+    return DUO_OK;
+}
+
+duo_status duo_cache_seq_lens(const duo_cache* c, int32_t layer, int64_t* lens) {
+    if (!c || !lens || layer < 0 || layer >= c->lay.num_layers) return DUO_ERR_INVALID_ARG;
+    const int64_t* L = seq_lens(c, layer);
+    for (int32_t b = 0; b < c->lay.batch; ++b) lens[b] = L[b];
+    return DUO_OK;
+}
+
+duo_status duo_cache_set_seq_lens(duo_cache* c, int32_t layer, const int64_t* lens) {
+    if (!c || !lens || layer < 0 || layer >= c->lay.num_layers) return DUO_ERR_INVALID_ARG;
+    for (int32_t b = 0; b < c->lay.batch; ++b)
+        if (lens[b] < 0 || lens[b] > c->lay.max_len) return DUO_ERR_INVALID_ARG;
+    int64_t* L = seq_lens(c, layer);
+    for (int32_t b = 0; b < c->lay.batch; ++b) L[b] = lens[b];
     return DUO_OK;
 }
 
@@ -288,31 +308,68 @@ duo_status duo_cache_error(duo_cache* c, void* stream, uint32_t* flags) {
     return DUO_OK;
 }
 
-duo_status duo_cache_append(duo_cache* c, int32_t layer, const void* k, const void* v, int64_t n_tok, void* stream) {
+namespace {
+
+// Append rows [0, n_tok[b]) of sequence b (k, v: [batch][max_tok][Hkv][D]).
+duo_status append_impl(duo_cache* c, int32_t layer, const void* k, const void* v, const int64_t* n_tok,
+                       int64_t max_tok, void* stream) {
     duo_status st = check_call(c, layer);
     if (st != DUO_OK) return st;
-    if (n_tok < 0) return DUO_ERR_INVALID_ARG;
-    if (n_tok == 0) return DUO_OK;
+    if (max_tok < 0) return DUO_ERR_INVALID_ARG;
+    const int32_t B = c->lay.batch;
+    int64_t* L = seq_lens(c, layer);
+    bool uniform = true, any = false;
+    for (int32_t b = 0; b < B; ++b) {
+        if (n_tok[b] < 0 || n_tok[b] > max_tok) return DUO_ERR_INVALID_ARG;
+        if (L[b] + n_tok[b] > c->lay.max_len) return DUO_ERR_CAPACITY;
+        uniform = uniform && L[b] == L[0] && n_tok[b] == n_tok[0];
+        any = any || n_tok[b] > 0;
+    }
+    if (!any) return DUO_OK;
     if (!k || !v) return DUO_ERR_INVALID_ARG;
     if (!aligned16(k) || !aligned16(v)) return DUO_ERR_ALIGNMENT;
-    if (c->len[layer] + n_tok > c->lay.max_len) return DUO_ERR_CAPACITY;
+    uniform = uniform && max_tok == n_tok[0];  // else the launch carries the row stride and counts
+    if (!uniform && B > kMaxRaggedBatch) return DUO_ERR_STATE;
     AppendParams p{};
     p.k = static_cast<const bf16*>(k);
     p.v = static_cast<const bf16*>(v);
     p.pools = c->pools;
-    p.len = c->len[layer];
-    p.n = n_tok;
+    p.len = L[0];
+    p.n = max_tok;
     p.max_len = c->lay.max_len;
-    p.B = c->lay.batch;
+    p.B = B;
     p.Hkv = c->lay.num_kv_heads;
     p.D = c->lay.head_dim;
     p.S = c->lay.sink;
     p.R = c->lay.recent;
     p.W = c->W;
+    p.num_sms = c->num_sms;
+    p.ragged = uniform ? 0 : 1;
+    if (!uniform) {
+        for (int32_t b = 0; b < B; ++b) {
+            p.seq_len[b] = L[b];
+            p.seq_n[b] = n_tok[b];
+        }
+    }
     fill_heads(c, layer, &p.heads);
     if (launch_append(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUO_ERR_CUDA;
-    c->len[layer] += n_tok;
+    for (int32_t b = 0; b < B; ++b) L[b] += n_tok[b];
     return DUO_OK;
+}
+
+}  // namespace
+
+duo_status duo_cache_append(duo_cache* c, int32_t layer, const void* k, const void* v, int64_t n_tok, void* stream) {
+    if (!c || layer < 0 || layer >= c->lay.num_layers) return DUO_ERR_INVALID_ARG;
+    if (n_tok < 0) return DUO_ERR_INVALID_ARG;
+    std::vector<int64_t> n(static_cast<size_t>(c->lay.batch), n_tok);
+    return append_impl(c, layer, k, v, n.data(), n_tok, stream);
+}
+
+duo_status duo_cache_append_ragged(duo_cache* c, int32_t layer, const void* k, const void* v, const int64_t* n_tok,
+                                   int64_t max_tok, void* stream) {
+    if (!c || !n_tok || layer < 0 || layer >= c->lay.num_layers) return DUO_ERR_INVALID_ARG;
+    return append_impl(c, layer, k, v, n_tok, max_tok, stream);
 }
 
 duo_status duo_prefill(duo_cache* c, int32_t layer, const void* q, const void* k, const void* v, void* out,
@@ -323,12 +380,15 @@ duo_status duo_prefill(duo_cache* c, int32_t layer, const void* q, const void* k
     if (n_tok == 0) return DUO_OK;
     if (!q || !k || !v || !out) return DUO_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DUO_ERR_ALIGNMENT;
-    if (c->len[layer] + n_tok > c->lay.max_len) return DUO_ERR_CAPACITY;
+    bool uniform = true;
+    const int64_t len0 = longest_seq(c, layer, &uniform);
+    if (!uniform) return DUO_ERR_STATE;  // chunked prefill of a ragged batch is not supported
+    if (len0 + n_tok > c->lay.max_len) return DUO_ERR_CAPACITY;
     const duo_layout& L = c->lay;
     PrefillParams p{};
     p.out = static_cast<bf16*>(out);
     p.err = c->err;
-    p.len = c->len[layer];
+    p.len = len0;
     p.C = static_cast<int32_t>(n_tok);
     p.B = L.batch;
     p.Hq = L.num_q_heads;
@@ -369,19 +429,21 @@ duo_status duo_decode(duo_cache* c, int32_t layer, const void* q, const void* k_
     if (st != DUO_OK) return st;
     if (!q || !k_new || !v_new || !out) return DUO_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return DUO_ERR_ALIGNMENT;
-    if (c->len[layer] + 1 > c->lay.max_len) return DUO_ERR_CAPACITY;
     DecodeParams p = c->decode_tmpl[layer];
+    st = fill_decode_lengths(c, layer, p);
+    if (st != DUO_OK) return st;
+    if (p.len + 1 > c->lay.max_len) return DUO_ERR_CAPACITY;
     p.q = static_cast<const bf16*>(q);
     p.k_new = static_cast<const bf16*>(k_new);
     p.v_new = static_cast<const bf16*>(v_new);
     p.out = static_cast<bf16*>(out);
-    p.len = c->len[layer];
     const int64_t rows = p.len + 1;
     const int64_t nsplit = decode_plan(c, layer, rows);
     p.split_rows = (rows + nsplit - 1) / nsplit;
     p.nsplit = static_cast<int32_t>((rows + p.split_rows - 1) / p.split_rows);
     if (launch_decode(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUO_ERR_CUDA;
-    c->len[layer] += 1;
+    int64_t* L = seq_lens(c, layer);
+    for (int32_t b = 0; b < c->lay.batch; ++b) L[b] += 1;
     return DUO_OK;
 }
 

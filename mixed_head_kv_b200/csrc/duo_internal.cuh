@@ -63,16 +63,24 @@ struct Pools {
     bf16* sv;
 };
 
+// Sequences of a batch may have different lengths (ragged batches) when the
+// batch has at most this many sequences; their lengths travel in the launch.
+constexpr int kMaxRaggedBatch = DUO_MAX_RAGGED_BATCH;
+
 // ------------------------------------------------------------------ append
 struct AppendParams {
     const bf16* k;  // [B][n][Hkv][D]
     const bf16* v;
     Pools pools;
-    int64_t len;      // tokens cached before this call
-    int64_t n;        // tokens appended
+    int64_t len;      // tokens cached before this call (uniform batch)
+    int64_t n;        // tokens appended (uniform batch); rows per sequence of k and v
     int64_t max_len;
     int32_t B, Hkv, D, S, R, W;
+    int32_t num_sms;
+    int32_t ragged;   // 1: per-sequence seq_len / seq_n below
     HeadMap heads;
+    int64_t seq_len[kMaxRaggedBatch];  // tokens cached before this call, per sequence
+    int64_t seq_n[kMaxRaggedBatch];    // tokens appended, per sequence (<= n)
 };
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s);
 
@@ -126,6 +134,7 @@ struct DecodeParams {
     uint32_t* counters;  // [B*Hkv] splits finished, reset by the merging CTA
     uint32_t* err;
     int64_t len;        // tokens cached before this step; the new token sits at position len
+                        // (uniform batch; the longest sequence when ragged)
     int64_t max_len;
     int64_t split_rows;  // rows per retrieval split
     int32_t nsplit;      // splits per retrieval (b, kv head)
@@ -135,6 +144,8 @@ struct DecodeParams {
     int16_t retr_list[DUO_MAX_KV_HEADS];
     int16_t strm_list[DUO_MAX_KV_HEADS];
     HeadMap heads;
+    int32_t ragged;                     // 1: per-sequence lengths in seq_len
+    int64_t seq_len[kMaxRaggedBatch];   // tokens cached before this step, per sequence
 };
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
 
@@ -178,7 +189,7 @@ struct duo_cache {
     int num_sms = 148;
     std::vector<uint8_t> is_retr;       // [layers][Hkv]
     std::vector<int32_t> pool_idx;      // [layers][Hkv] dense index within its pool
-    std::vector<int64_t> len;           // [layers]
+    std::vector<int64_t> len;           // [layers][batch] tokens cached per sequence
     int64_t n_retr_all = 0, n_strm_all = 0;
     duo::Pools pools{};
     float* part_o = nullptr;
@@ -190,6 +201,41 @@ struct duo_cache {
     std::vector<int64_t> plan_key;               // [layers] rows / 256 of the cached split plan
     std::vector<int64_t> plan_nsplit;            // [layers] the plan's split count
 };
+
+// Per-sequence lengths of one layer ([batch] host values).
+inline int64_t* seq_lens(duo_cache* c, int32_t layer) {
+    return c->len.data() + static_cast<size_t>(layer) * c->lay.batch;
+}
+inline const int64_t* seq_lens(const duo_cache* c, int32_t layer) {
+    return c->len.data() + static_cast<size_t>(layer) * c->lay.batch;
+}
+
+// Longest sequence of a layer, and whether all sequences have that length.
+inline int64_t longest_seq(const duo_cache* c, int32_t layer, bool* uniform) {
+    const int64_t* L = seq_lens(c, layer);
+    int64_t mx = L[0];
+    bool uni = true;
+    for (int32_t b = 1; b < c->lay.batch; ++b) {
+        if (L[b] > mx) mx = L[b];
+        uni = uni && (L[b] == L[0]);
+    }
+    if (uniform) *uniform = uni;
+    return mx;
+}
+
+// Lengths of a decode step: the longest sequence in p.len and, for a ragged
+// batch, every sequence's length. DUO_ERR_STATE if a ragged batch is larger
+// than the launch can carry.
+inline duo_status fill_decode_lengths(const duo_cache* c, int32_t layer, duo::DecodeParams& p) {
+    bool uniform = true;
+    p.len = longest_seq(c, layer, &uniform);
+    p.ragged = uniform ? 0 : 1;
+    if (uniform) return DUO_OK;
+    if (c->lay.batch > duo::kMaxRaggedBatch) return DUO_ERR_STATE;
+    const int64_t* L = seq_lens(c, layer);
+    for (int32_t b = 0; b < c->lay.batch; ++b) p.seq_len[b] = L[b];
+    return DUO_OK;
+}
 
 // Split count for a decode step over `rows` keys of `layer`. The plan is kept
 // per layer and recomputed when rows / 256 changes: any split count is
