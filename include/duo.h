@@ -157,10 +157,22 @@ DUO_API duo_status duo_cache_append_ragged(duo_cache* cache, int32_t layer, cons
  * streaming heads over the sinks and the recent window, read from the
  * streaming cache for positions < len and from k/v for the chunk.
  * Does NOT modify the cache: call duo_cache_append(layer, k, v, n_tok) after it.
- * All sequences must have the same length (DUO_ERR_STATE otherwise).
- * DUO_ERR_CAPACITY if a retrieval head could not hold len + n_tok tokens. */
+ * Each sequence's chunk starts at its own length len_b (a ragged batch needs
+ * batch <= DUO_MAX_RAGGED_BATCH, else DUO_ERR_STATE).
+ * DUO_ERR_CAPACITY if a retrieval head could not hold len_b + n_tok tokens. */
 DUO_API duo_status duo_prefill(duo_cache* cache, int32_t layer, const void* q, const void* k, const void* v, void* out,
                        int64_t n_tok, void* stream);
+
+/* duo_prefill_ragged — duo_prefill with a different chunk length per sequence.
+ *   q, k, v, out  as duo_prefill with max_tok rows per sequence; sequence b's
+ *                 rows [0, n_tok[b]) are its chunk at positions
+ *                 [len_b, len_b + n_tok[b]); its other rows are not read and its
+ *                 other output rows are not written
+ *   n_tok         host [batch], 0 <= n_tok[b] <= max_tok
+ * Follow it with duo_cache_append_ragged(layer, k, v, n_tok, max_tok). Needs
+ * batch <= DUO_MAX_RAGGED_BATCH unless all lengths and counts are equal. */
+DUO_API duo_status duo_prefill_ragged(duo_cache* cache, int32_t layer, const void* q, const void* k, const void* v,
+                              void* out, const int64_t* n_tok, int64_t max_tok, void* stream);
 
 /* duo_decode — one decoding step of `layer` (DuoAttention decoding).
  *   q            device [batch][num_q_heads][head_dim], sequence b's query at

@@ -42,7 +42,7 @@ DUO_MAX_RAGGED_BATCH = 64  # sequences of different lengths per batch (include/d
 EXPORTED = ("duo_cache_alloc", "duo_cache_free", "duo_cache_append", "duo_prefill", "duo_decode",
             "duo_cache_len", "duo_cache_set_len", "duo_cache_views", "duo_cache_error", "duo_status_str",
             "duo_decode_static_scratch", "duo_cache_append_ragged", "duo_cache_seq_lens",
-            "duo_cache_set_seq_lens")
+            "duo_cache_set_seq_lens", "duo_prefill_ragged")
 
 
 class duo_layout(ctypes.Structure):
@@ -81,6 +81,8 @@ _lib.duo_cache_views.argtypes = [_P, _I32, _I32, ctypes.POINTER(_P), ctypes.POIN
                                  ctypes.POINTER(_I32)]
 _lib.duo_cache_append_ragged.restype = _ST
 _lib.duo_cache_append_ragged.argtypes = [_P, _I32, _P, _P, ctypes.POINTER(_I64), _I64, _P]
+_lib.duo_prefill_ragged.restype = _ST
+_lib.duo_prefill_ragged.argtypes = [_P, _I32, _P, _P, _P, _P, ctypes.POINTER(_I64), _I64, _P]
 _lib.duo_cache_seq_lens.restype = _ST
 _lib.duo_cache_seq_lens.argtypes = [_P, _I32, ctypes.POINTER(_I64)]
 _lib.duo_cache_set_seq_lens.restype = _ST
@@ -186,6 +188,13 @@ def duo_cache_append_ragged(handle, layer, k, v, n_tok: Sequence[int], max_tok: 
                                         _stream(stream) if k is not None else None)
 
 
+def duo_prefill_ragged(handle, layer, q, k, v, out, n_tok: Sequence[int], max_tok: int, stream=None) -> int:
+    """Sequence b's chunk is rows [0, n_tok[b]) of q/k/v [batch][max_tok][H][D]."""
+    n = (_I64 * max(1, len(n_tok)))(*[int(x) for x in n_tok])
+    return _lib.duo_prefill_ragged(handle, layer, _ptr(q), _ptr(k), _ptr(v), _ptr(out), n, max_tok,
+                                   _stream(stream) if q is not None else None)
+
+
 def duo_cache_seq_lens(handle, layer, batch: int):
     lens = (_I64 * batch)()
     st = _lib.duo_cache_seq_lens(handle, layer, lens)
@@ -247,6 +256,9 @@ class DuoCache:
         """Per-sequence token counts n_tok[b] <= k.shape[1] (rows past them are not read)."""
         _check(duo_cache_append_ragged(self.handle, layer, k, v, n_tok, k.shape[1], stream),
                "duo_cache_append_ragged")
+
+    def prefill_ragged(self, layer, q, k, v, out, n_tok, stream=None):
+        _check(duo_prefill_ragged(self.handle, layer, q, k, v, out, n_tok, q.shape[1], stream), "duo_prefill_ragged")
 
     def seq_lens(self, layer):
         st, lens = duo_cache_seq_lens(self.handle, layer, self.layout.batch)

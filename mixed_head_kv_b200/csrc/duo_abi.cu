@@ -372,24 +372,43 @@ duo_status duo_cache_append_ragged(duo_cache* c, int32_t layer, const void* k, c
     return append_impl(c, layer, k, v, n_tok, max_tok, stream);
 }
 
-duo_status duo_prefill(duo_cache* c, int32_t layer, const void* q, const void* k, const void* v, void* out,
-                       int64_t n_tok, void* stream) {
+namespace {
+
+// Prefill of sequence b's chunk rows [0, n_tok[b]) at its own length (q, k, v,
+// out: [batch][max_tok][H][D]).
+duo_status prefill_impl(duo_cache* c, int32_t layer, const void* q, const void* k, const void* v, void* out,
+                        const int64_t* n_tok, int64_t max_tok, void* stream) {
     duo_status st = check_call(c, layer);
     if (st != DUO_OK) return st;
-    if (n_tok < 0 || n_tok > (int64_t{1} << 30)) return DUO_ERR_INVALID_ARG;
-    if (n_tok == 0) return DUO_OK;
+    if (max_tok < 0 || max_tok > (int64_t{1} << 30)) return DUO_ERR_INVALID_ARG;
+    const int32_t B = c->lay.batch;
+    const int64_t* lens = seq_lens(c, layer);
+    bool uniform = true, any = false;
+    for (int32_t b = 0; b < B; ++b) {
+        if (n_tok[b] < 0 || n_tok[b] > max_tok) return DUO_ERR_INVALID_ARG;
+        if (lens[b] + n_tok[b] > c->lay.max_len) return DUO_ERR_CAPACITY;
+        uniform = uniform && lens[b] == lens[0] && n_tok[b] == max_tok;
+        any = any || n_tok[b] > 0;
+    }
+    if (!any) return DUO_OK;
     if (!q || !k || !v || !out) return DUO_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DUO_ERR_ALIGNMENT;
-    bool uniform = true;
-    const int64_t len0 = longest_seq(c, layer, &uniform);
-    if (!uniform) return DUO_ERR_STATE;  // chunked prefill of a ragged batch is not supported
-    if (len0 + n_tok > c->lay.max_len) return DUO_ERR_CAPACITY;
+    if (!uniform && B > kMaxRaggedBatch) return DUO_ERR_STATE;
+    const int64_t n_rows = max_tok;  // rows per sequence of the padded tensors
+    const int64_t len0 = lens[0];
     const duo_layout& L = c->lay;
     PrefillParams p{};
     p.out = static_cast<bf16*>(out);
     p.err = c->err;
     p.len = len0;
-    p.C = static_cast<int32_t>(n_tok);
+    p.C = static_cast<int32_t>(n_rows);
+    p.ragged = uniform ? 0 : 1;
+    if (!uniform) {
+        for (int32_t b = 0; b < B; ++b) {
+            p.seq_len[b] = lens[b];
+            p.seq_c[b] = static_cast<int32_t>(n_tok[b]);
+        }
+    }
     p.B = L.batch;
     p.Hq = L.num_q_heads;
     p.Hkv = L.num_kv_heads;
@@ -398,7 +417,7 @@ duo_status duo_prefill(duo_cache* c, int32_t layer, const void* q, const void* k
     p.S = L.sink;
     p.R = L.recent;
     p.W = c->W;
-    p.n_qt = static_cast<int32_t>((n_tok + kTileQ - 1) / kTileQ);
+    p.n_qt = static_cast<int32_t>((n_rows + kTileQ - 1) / kTileQ);
     p.scale_log2 = c->scale * 1.4426950408889634f;
     fill_heads(c, layer, &p.heads);
     int nq = 0;
@@ -415,12 +434,28 @@ duo_status duo_prefill(duo_cache* c, int32_t layer, const void* q, const void* k
     maps.rv = c->map_rv;
     maps.sk = c->map_sk;
     maps.sv = c->map_sv;
-    if (!make_chunk_map(&maps.q, q, L.head_dim, L.num_q_heads, n_tok, L.batch) ||
-        !make_chunk_map(&maps.k, k, L.head_dim, L.num_kv_heads, n_tok, L.batch) ||
-        !make_chunk_map(&maps.v, v, L.head_dim, L.num_kv_heads, n_tok, L.batch))
+    if (!make_chunk_map(&maps.q, q, L.head_dim, L.num_q_heads, n_rows, L.batch) ||
+        !make_chunk_map(&maps.k, k, L.head_dim, L.num_kv_heads, n_rows, L.batch) ||
+        !make_chunk_map(&maps.v, v, L.head_dim, L.num_kv_heads, n_rows, L.batch))
         return DUO_ERR_CUDA;
     if (launch_prefill(p, maps, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUO_ERR_CUDA;
     return DUO_OK;
+}
+
+}  // namespace
+
+duo_status duo_prefill(duo_cache* c, int32_t layer, const void* q, const void* k, const void* v, void* out,
+                       int64_t n_tok, void* stream) {
+    if (!c || layer < 0 || layer >= c->lay.num_layers) return DUO_ERR_INVALID_ARG;
+    if (n_tok < 0) return DUO_ERR_INVALID_ARG;
+    std::vector<int64_t> n(static_cast<size_t>(c->lay.batch), n_tok);
+    return prefill_impl(c, layer, q, k, v, out, n.data(), n_tok, stream);
+}
+
+duo_status duo_prefill_ragged(duo_cache* c, int32_t layer, const void* q, const void* k, const void* v, void* out,
+                              const int64_t* n_tok, int64_t max_tok, void* stream) {
+    if (!c || !n_tok || layer < 0 || layer >= c->lay.num_layers) return DUO_ERR_INVALID_ARG;
+    return prefill_impl(c, layer, q, k, v, out, n_tok, max_tok, stream);
 }
 
 duo_status duo_decode(duo_cache* c, int32_t layer, const void* q, const void* k_new, const void* v_new, void* out,

@@ -156,14 +156,17 @@ constexpr int kTileK = 128;   // keys per KV tile
 struct PrefillParams {
     bf16* out;  // [B][C][Hq][D]
     uint32_t* err;
-    int64_t len;  // tokens cached before the chunk
-    int32_t C;    // chunk length
+    int64_t len;  // tokens cached before the chunk (uniform batch)
+    int32_t C;    // chunk length; rows per sequence of q, k, v and out
     int32_t B, Hq, Hkv, G, D, S, R, W;
     int32_t n_qt;      // ceil(C / kTileQ)
     int32_t n_retr_q;  // retrieval query heads (listed first in qhead)
     float scale_log2;
     int16_t qhead[DUO_MAX_Q_HEADS];
     HeadMap heads;
+    int32_t ragged;                    // 1: per-sequence seq_len / seq_c below
+    int64_t seq_len[kMaxRaggedBatch];  // tokens cached before the chunk, per sequence
+    int32_t seq_c[kMaxRaggedBatch];    // chunk rows that are tokens, per sequence (<= C)
 };
 
 struct PrefillMaps {

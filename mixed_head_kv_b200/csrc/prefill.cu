@@ -91,6 +91,8 @@ constexpr uint32_t kTmemP = 32;   // P of a key tile at its S buffer + 32 (64 co
 // What one work item attends to.
 struct Item {
     int b, head, g, qt, retr, pool;
+    int64_t L;    // the sequence's cache length (tokens before its chunk)
+    int C;        // the sequence's chunk length (rows of the padded chunk that are tokens)
     int q0;       // first chunk row of the query tile
     int n_cache;  // cache tiles
     int src_cache;
@@ -120,7 +122,13 @@ __device__ __forceinline__ Item make_item(const PrefillParams& p) {
     it.retr = p.heads.is_retr[it.g];
     it.pool = p.heads.pool_idx[it.g];
     it.q0 = it.qt * kTileQ;
-    const int64_t L = p.len;
+    it.L = p.ragged ? p.seq_len[it.b] : p.len;
+    it.C = p.ragged ? p.seq_c[it.b] : p.C;
+    if (it.q0 >= it.C) {  // a query tile past this sequence's chunk (ragged batch): no work
+        it.n_tiles = 0;
+        return it;
+    }
+    const int64_t L = it.L;
     if (it.retr) {
         it.src_cache = 0;
         it.n_cache = static_cast<int>((L + kTileK - 1) / kTileK);
@@ -137,7 +145,7 @@ __device__ __forceinline__ Item make_item(const PrefillParams& p) {
         it.n_cache = static_cast<int>((slots + kTileK - 1) / kTileK);
         int a = 0;
         if (L < p.S) {
-            const int64_t sink_rows = (p.S - L < p.C) ? (p.S - L) : p.C;
+            const int64_t sink_rows = (p.S - L < it.C) ? (p.S - L) : it.C;
             a = static_cast<int>((sink_rows + kTileK - 1) / kTileK);
             if (a > it.qt + 1) a = it.qt + 1;
         }
@@ -189,11 +197,11 @@ struct RingVis {
     int64_t a0, b0, a1, b1;
 };
 
-__device__ __forceinline__ RingVis ring_visible(const PrefillParams& p, int qrow) {
+__device__ __forceinline__ RingVis ring_visible(const PrefillParams& p, int64_t len, int qrow) {
     RingVis g{0, 0, 0, 0};
-    int64_t lo = p.len + qrow - p.R + 1;
+    int64_t lo = len + qrow - p.R + 1;
     if (lo < p.S) lo = p.S;
-    const int64_t c = p.len - lo;
+    const int64_t c = len - lo;
     if (c > 0) {
         const int64_t r0 = (lo - p.S) % p.R;
         g.a0 = p.S + r0;
@@ -215,13 +223,14 @@ __device__ __forceinline__ RingVis ring_visible(const PrefillParams& p, int qrow
 //     j < len; ring slots as in ring_visible.
 //   src 2 (chunk): row c is position len + c, valid for c < C, causal, and for
 //     streaming heads a sink (len + c < sink) or inside the window.
-__device__ __forceinline__ uint32_t visible_bits(const PrefillParams& p, int retr, int src, int row0, int w,
+__device__ __forceinline__ uint32_t visible_bits(const PrefillParams& p, const Item& it, int src, int row0, int w,
                                                  int qrow, const RingVis& ring) {
-    const int64_t L = p.len;
+    const int64_t L = it.L;
+    const int retr = it.retr;
     const int base = row0 + 32 * w;
     if (src == 0) return bits_below(L - base);
     if (src == 2) {
-        const int hi = (qrow < p.C - 1 ? qrow : p.C - 1);
+        const int hi = (qrow < it.C - 1 ? qrow : it.C - 1);
         const uint32_t causal = bits_below(static_cast<int64_t>(hi) + 1 - base);
         if (retr) return causal;
         const uint32_t sink = bits_below(static_cast<int64_t>(p.S) - L - base);
@@ -274,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const Item it = make_item(p);
+    if (it.n_tiles == 0) return;  // uniform over the CTA, before any barrier or TMEM use
 
     if (tid == 0) {
         mbar_init(bar(kQFull), 1);
@@ -411,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qrow = it.q0 + row;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t tO = tmem + lane_base + kTmemO + h * D;
-        const RingVis ring = ring_visible(p, qrow);
+        const RingVis ring = ring_visible(p, it.L, qrow);
         const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
         volatile float* xm = xchg;        // [half][row] running max
         volatile float* xl = xchg + 256;  // [half][row] row sum
@@ -441,11 +451,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             int src, row0;
             tile_of(it, j, src, row0);
             const bool full =
-                it.retr && ((src == 0 && row0 + kTileK <= p.len) || (src == 2 && row0 + kTileK <= it.q0));
+                it.retr && ((src == 0 && row0 + kTileK <= it.L) || (src == 2 && row0 + kTileK <= it.q0));
             if (!full) {
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
-                    const uint32_t bits = visible_bits(p, it.retr, src, row0, 2 * h + w, qrow, ring);
+                    const uint32_t bits = visible_bits(p, it, src, row0, 2 * h + w, qrow, ring);
 #pragma unroll
                     for (int k = 0; k < 32; ++k)
                         if (!((bits >> k) & 1u)) s[w * 32 + k] = -INFINITY;
@@ -532,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(tO0 + c * 32, r0);
                 tmem_ld32(tO0 + D + c * 32, r1);
                 tc_wait_ld();
-                if (qrow < p.C) {
+                if (qrow < it.C) {
 #pragma unroll
                     for (int v8 = 0; v8 < 4; ++v8) {
                         uint32_t w[4];

@@ -112,7 +112,8 @@ def test_ragged_state_rules(duo):
     assert st == duo.DUO_ERR_STATE  # no single length
     q = torch.zeros((2, 8, 4, 64), dtype=torch.bfloat16, device="cuda")
     o = torch.empty_like(q)
-    assert duo.duo_prefill(cache.handle, 0, q, q, q, o, 8) == duo.DUO_ERR_STATE
+    assert duo.duo_prefill_ragged(cache.handle, 0, q, q, q, o, [9, 1], 8) == duo.DUO_ERR_INVALID_ARG
+    assert duo.duo_prefill_ragged(cache.handle, 0, q, q, q, o, [8, 8], 8) == duo.DUO_OK  # 18, 28 <= 64
     kv = torch.zeros((2, 50, 4, 64), dtype=torch.bfloat16, device="cuda")
     # capacity is checked per sequence, before anything is written
     assert duo.duo_cache_append_ragged(cache.handle, 0, kv, kv, [40, 50], 50) == duo.DUO_ERR_CAPACITY
@@ -135,3 +136,54 @@ def test_ragged_batch_limit(duo):
     cache.set_length(0, 5)  # uniform lengths work at any batch size
     assert duo.duo_decode(cache.handle, 0, x, x, x, torch.empty_like(x)) == duo.DUO_OK
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("G,lens,n_tok", [
+    (1, [100, 37, 260], [50, 129, 7]),   # the third sequence's second query tile is empty
+    (2, [0, 300, 3], [200, 1, 130]),     # a fresh sequence, a one-token chunk, a chunk over the sinks
+])
+def test_ragged_prefill_then_decode(duo, G, lens, n_tok):
+    Hkv = 4
+    w = make_workload(B=len(lens), Hq=Hkv * G, Hkv=Hkv, D=64, S=4, R=64, mask=[1, 0, 1, 0])
+    B, steps = w.batch, 3
+    T = max(l + n for l, n in zip(lens, n_tok)) + steps + 1
+    q, k, v = workloads.tokens(w, 0, 0, T)
+    mask = workloads.retrieval_mask(w)
+    cache = duo.DuoCache(1, B, w.num_q_heads, w.num_kv_heads, w.head_dim, w.sink, w.recent, T + 8, mask)
+
+    def padded(x, starts, counts, rows):
+        out = torch.zeros((B, rows) + tuple(x.shape[2:]), dtype=torch.bfloat16)
+        for b in range(B):
+            out[b, :counts[b]] = x[b, starts[b]:starts[b] + counts[b]]
+        return out.cuda()
+
+    mx = max(max(lens), 1)
+    cache.append_ragged(0, padded(k, [0] * B, lens, mx), padded(v, [0] * B, lens, mx), lens)
+    C = max(n_tok)
+    qc, kc, vc = (padded(x, lens, n_tok, C) for x in (q, k, v))
+    out = torch.full_like(qc, float("nan"))
+    cache.prefill_ragged(0, qc, kc, vc, out, n_tok)
+    cache.append_ragged(0, kc, vc, n_tok)
+    torch.cuda.synchronize()
+    assert cache.error_flags() == 0
+    out = out.cpu()
+    for b in range(B):
+        pos = np.arange(lens[b], lens[b] + n_tok[b])
+        if len(pos):
+            ref = oracle.attention(q[b:b + 1, pos].permute(0, 2, 1, 3), pos,
+                                   k[b:b + 1, :pos[-1] + 1].permute(0, 2, 1, 3),
+                                   v[b:b + 1, :pos[-1] + 1].permute(0, 2, 1, 3), mask, w.sink, w.recent)
+            assert_close(out[b, :n_tok[b]], ref[0].transpose(1, 0, 2), f"seq {b} prefill")
+        assert torch.isnan(out[b, n_tok[b]:].float()).all(), f"seq {b}: rows past its chunk were written"
+    base = [l + n for l, n in zip(lens, n_tok)]
+    assert cache.seq_lens(0) == base
+    for t in range(steps):
+        rows = [base[b] + t for b in range(B)]
+        qd, kd, vd = (torch.stack([x[b, rows[b]] for b in range(B)]).cuda() for x in (q, k, v))
+        o = torch.full_like(qd, float("nan"))
+        cache.decode(0, qd, kd, vd, o)
+        o = o.cpu()
+        for b in range(B):
+            assert_close(o[b], _oracle_decode(w, q, k, v, b, rows[b]), f"seq {b} decode {t}")
+    for b in range(B):
+        _check_seq_cache(cache, w, b, k, v, base[b] + steps)
