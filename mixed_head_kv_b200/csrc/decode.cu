@@ -12,7 +12,8 @@
 // len - recent, which is outside the new query's window.
 //
 // Memory path: each of the 4 warps streams a contiguous part of the item's
-// rows through its own 3-stage ring in shared memory, filled by bulk async
+// rows through its own ring in shared memory (3 stages; 2 for query groups of
+// 2 and 4, which run three CTAs per SM), filled by bulk async
 // copies (cp.async.bulk, one K block and one V block of 4 KB per stage,
 // completion on an mbarrier). Each K/V row is read from HBM exactly once and
 // serves all G query heads of its group. A row of D bf16 is consumed by D/8

@@ -16,7 +16,7 @@
  * For GQA models the head type belongs to the KV head and every query head of
  * its group inherits it.
  *
- * Readings of points the pages leave open (each is listed in the design doc):
+ * Readings of points the pages leave open:
  *   - key set of a streaming head for a query at absolute position p:
  *       K(p) = { j <= p : j < sink  or  p - j < recent }
  *     ("recent" counts the query's own token; the union counts a key once);
