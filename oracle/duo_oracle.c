@@ -48,8 +48,8 @@ static double bf16_to_double(uint16_t h) {
 
 /* Membership of key position j in the key set of a query at position p.
  * Retrieval head: every previous token. Streaming head: attention sinks plus
- * the recent window (abstract: streaming heads "focus on recent tokens and
- * attention sinks" with a constant-length cache). */
+ * the recent window (DuoAttention abstract: a streaming head keeps only the
+ * sink tokens and the latest tokens, in a cache of fixed size). */
 int duo_oracle_key_allowed(int is_retrieval, int64_t p, int64_t j, int64_t sink, int64_t recent) {
     if (j < 0 || j > p) return 0;
     if (is_retrieval) return 1;

@@ -4,7 +4,7 @@
 - special cases that reduce to a library routine (PyTorch's causal and masked
   scaled_dot_product_attention in float64);
 - an evict-oldest cache simulation (a second derivation of the streaming key
-  set from the "constant-length cache of sinks + recent tokens" statement);
+  set from the abstract's fixed-size cache of sink and latest tokens);
 - closed forms, invariants and exact special cases.
 """
 import json
