@@ -40,6 +40,7 @@
 // the MMA reads them through descriptors). Every mbarrier wait is time-bounded;
 // on timeout the CTA records kErrPrefillWait and unwinds.
 #include "duo_internal.cuh"
+#include "mask_rules.cuh"
 #include "sm100.cuh"
 
 namespace duo {
@@ -175,70 +176,14 @@ __device__ __forceinline__ void record_abort(uint32_t* err, volatile int* abort_
     atomicOr(err, kErrPrefillWait);
 }
 
-// Bits k of a 32-bit word set for k < x (x clamped to [0, 32]).
-__device__ __forceinline__ uint32_t bits_below(int64_t x) {
-    if (x <= 0) return 0u;
-    if (x >= 32) return 0xFFFFFFFFu;
-    return (1u << static_cast<uint32_t>(x)) - 1u;
-}
-
-// Bits k of a 32-bit word set for base + k in [lo, hi).
-__device__ __forceinline__ uint32_t bits_in(int64_t lo, int64_t hi, int64_t base) {
-    return bits_below(hi - base) & ~bits_below(lo - base);
-}
-
-// Ring slots of the streaming cache visible from one query row, as at most two
-// slot ranges [a0, b0) and [a1, b1). The ring holds the latest min(recent,
-// len - sink) positions p >= sink below len, position p in slot
-// sink + (p - sink) mod recent; the query at len + qrow sees those with
-// p > len + qrow - recent, a contiguous run of positions [lo, len) that wraps
-// at most once in slot order.
-struct RingVis {
-    int64_t a0, b0, a1, b1;
-};
-
-__device__ __forceinline__ RingVis ring_visible(const PrefillParams& p, int64_t len, int qrow) {
-    RingVis g{0, 0, 0, 0};
-    int64_t lo = len + qrow - p.R + 1;
-    if (lo < p.S) lo = p.S;
-    const int64_t c = len - lo;
-    if (c > 0) {
-        const int64_t r0 = (lo - p.S) % p.R;
-        g.a0 = p.S + r0;
-        if (r0 + c <= p.R) {
-            g.b0 = p.S + r0 + c;
-        } else {
-            g.b0 = p.S + p.R;
-            g.a1 = p.S;
-            g.b1 = p.S + r0 + c - p.R;
-        }
-    }
-    return g;
-}
-
 // Visibility of keys [32w, 32w+32) of tile (src, row0) from chunk query row
-// `qrow` (absolute position len + qrow), one bit per key.
-//   src 0 (retrieval cache): slot j holds position j, valid for j < len.
-//   src 1 (streaming cache): sink slots j < sink hold position j, valid for
-//     j < len; ring slots as in ring_visible.
-//   src 2 (chunk): row c is position len + c, valid for c < C, causal, and for
-//     streaming heads a sink (len + c < sink) or inside the window.
+// `qrow`: src 0 retrieval cache, 1 streaming cache, 2 chunk (mask_rules.cuh).
 __device__ __forceinline__ uint32_t visible_bits(const PrefillParams& p, const Item& it, int src, int row0, int w,
                                                  int qrow, const RingVis& ring) {
-    const int64_t L = it.L;
-    const int retr = it.retr;
-    const int base = row0 + 32 * w;
-    if (src == 0) return bits_below(L - base);
-    if (src == 2) {
-        const int hi = (qrow < it.C - 1 ? qrow : it.C - 1);
-        const uint32_t causal = bits_below(static_cast<int64_t>(hi) + 1 - base);
-        if (retr) return causal;
-        const uint32_t sink = bits_below(static_cast<int64_t>(p.S) - L - base);
-        const uint32_t band = ~bits_below(static_cast<int64_t>(qrow) - p.R + 1 - base);
-        return causal & (sink | band);
-    }
-    const int64_t sink_hi = L < p.S ? L : p.S;
-    return bits_in(0, sink_hi, base) | bits_in(ring.a0, ring.b0, base) | bits_in(ring.a1, ring.b1, base);
+    const int64_t base = row0 + 32 * w;
+    if (src == 0) return retrieval_cache_bits(it.L, base);
+    if (src == 2) return chunk_bits(it.retr, it.L, it.C, p.S, p.R, qrow, base);
+    return streaming_cache_bits(it.L, p.S, ring, base);
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -421,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qrow = it.q0 + row;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t tO = tmem + lane_base + kTmemO + h * D;
-        const RingVis ring = ring_visible(p, it.L, qrow);
+        const RingVis ring = ring_visible(it.L, p.S, p.R, qrow);
         const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
         volatile float* xm = xchg;        // [half][row] running max
         volatile float* xl = xchg + 256;  // [half][row] row sum
