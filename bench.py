@@ -359,7 +359,40 @@ def load_traffic(kernel: str):
         return None
 
 
+def gpu_local_cpus(device):
+    """CPUs of the GPU's own NUMA node (sysfs, read only), within this process's
+    allowed set; None when unknown."""
+    try:
+        pr = torch.cuda.get_device_properties(device)
+        path = (f"/sys/bus/pci/devices/{pr.pci_domain_id:04x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0/"
+                "local_cpulist")
+        cpus = set()
+        for part in open(path).read().strip().split(","):
+            a, _, b = part.partition("-")
+            cpus.update(range(int(a), int(b or a) + 1))
+        cpus &= os.sched_getaffinity(0)
+        return cpus or None
+    except Exception:
+        return None
+
+
 def run_e2e(duo, step, args, sp, device):
+    """See run_e2e_on: the host thread runs on the GPU's NUMA node while the pinned
+    buffers are allocated and filled, so the copies read node-local memory."""
+    old = os.sched_getaffinity(0)
+    local = gpu_local_cpus(device)
+    if local:
+        os.sched_setaffinity(0, local)
+    try:
+        out = run_e2e_on(duo, step, args, sp, device)
+    finally:
+        if local:
+            os.sched_setaffinity(0, old)
+    out["host_cpus"] = len(local) if local else "unchanged"
+    return out
+
+
+def run_e2e_on(duo, step, args, sp, device):
     """The same step from pinned host buffers through the same C ABI: every input is
     copied host -> device and every output device -> host inside the timed region.
     Copies run on their own streams and overlap the kernels: the upload of chunk i+1
