@@ -50,6 +50,12 @@ def _load():
         lib.duo_oracle_key_allowed.restype = ctypes.c_int
         lib.duo_oracle_key_allowed.argtypes = [ctypes.c_int, i64, i64, i64, i64]
         lib.duo_oracle_num_threads.restype = ctypes.c_int
+        lib.duo_oracle_e4m3_value.restype = ctypes.c_double
+        lib.duo_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.duo_oracle_e4m3_code.restype = ctypes.c_uint8
+        lib.duo_oracle_e4m3_code.argtypes = [ctypes.c_double]
+        lib.duo_oracle_e4m3_quantize.restype = None
+        lib.duo_oracle_e4m3_quantize.argtypes = [P, i64, ctypes.c_float, P]
         _lib = lib
     return _lib
 
@@ -125,3 +131,21 @@ def slot_positions(is_retrieval: int, sink: int, recent: int, length: int, nslot
     pos = np.zeros(nslots, dtype=np.int64)
     lib.duo_oracle_slot_positions(int(is_retrieval), sink, recent, length, nslots, pos.ctypes.data)
     return pos
+
+
+def e4m3_value(code: int) -> float:
+    """Value of an FP8 E4M3 code (NaN for 0x7F / 0xFF)."""
+    return float(_load().duo_oracle_e4m3_value(int(code)))
+
+
+def e4m3_code(x: float) -> int:
+    """E4M3 code of x: nearest, ties to even, saturating to +-448."""
+    return int(_load().duo_oracle_e4m3_code(float(x)))
+
+
+def e4m3_quantize(x, inv_scale: float) -> np.ndarray:
+    """Codes of bf16 values x times inv_scale (product rounded to fp32 first)."""
+    xb = _bits(x)
+    out = np.zeros(xb.shape, dtype=np.uint8)
+    _load().duo_oracle_e4m3_quantize(xb.ctypes.data, xb.size, float(inv_scale), out.ctypes.data)
+    return out

@@ -187,3 +187,57 @@ int duo_oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------
+ * FP8 E4M3 retrieval caches (a next step of this library: the pages reach
+ * their longest contexts only together with KV quantization). Reading: each
+ * retrieval-head element x (bf16) is stored as the E4M3 code of x * inv_scale,
+ * the product taken in fp32 (inv_scale = the fp32 reciprocal of a per-head
+ * scale), rounded to nearest with ties to even and saturated to +-448; it is
+ * read back as value(code) * scale.
+ *
+ * E4M3 (the "fn" variant of the OCP 8-bit floating-point formats): 1 sign bit,
+ * 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds the
+ * subnormals m * 2^-9; exponent field 15 with mantissa 7 is NaN (no infinity);
+ * the largest finite magnitude is 1.75 * 2^8 = 448.
+ * ---------------------------------------------------------------------- */
+
+/* Value of an E4M3 code (NaN for 0x7F and 0xFF). */
+double duo_oracle_e4m3_value(uint8_t c) {
+    const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+/* E4M3 code of x: round to nearest, ties to even; magnitudes above 448
+ * (infinity included) saturate to 448; NaN gives 0x7F. */
+uint8_t duo_oracle_e4m3_code(double x) {
+    if (isnan(x)) return 0x7F;
+    const uint8_t s = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs(x);
+    if (a >= 448.0) return (uint8_t)(s | 0x7E);
+    int e = (int)floor(log2(a > 0.0 ? a : 1.0));
+    if (a == 0.0) return s;
+    if (e < -6) { /* subnormal: units of 2^-9 */
+        const double m = nearbyint(ldexp(a, 9)); /* default rounding mode: to nearest, ties to even */
+        return (uint8_t)(s | (int)m);           /* m == 8 is the smallest normal, code 0x08 */
+    }
+    /* guard against log2 rounding at exact powers of two */
+    if (ldexp(1.0, e) > a) --e;
+    if (ldexp(1.0, e + 1) <= a) ++e;
+    double m = nearbyint((ldexp(a, -e) - 1.0) * 8.0);
+    if (m == 8.0) { m = 0.0; ++e; }
+    if (e > 8 || (e == 8 && m > 6.0)) return (uint8_t)(s | 0x7E); /* rounded past 448 */
+    return (uint8_t)(s | ((e + 7) << 3) | (int)m);
+}
+
+/* Codes of n bf16 values times inv_scale, the product rounded to fp32 first. */
+void duo_oracle_e4m3_quantize(const uint16_t* x, int64_t n, float inv_scale, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) {
+        const float prod = (float)bf16_to_double(x[i]) * inv_scale;
+        out[i] = duo_oracle_e4m3_code((double)prod);
+    }
+}
