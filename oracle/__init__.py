@@ -54,6 +54,9 @@ def _load():
         lib.duo_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
         lib.duo_oracle_e4m3_code.restype = ctypes.c_uint8
         lib.duo_oracle_e4m3_code.argtypes = [ctypes.c_double]
+        lib.duo_oracle_attend_rows_e4m3.restype = ctypes.c_int
+        lib.duo_oracle_attend_rows_e4m3.argtypes = [P, P, P, i64, ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                                    ctypes.c_double, P, P]
         lib.duo_oracle_e4m3_quantize.restype = None
         lib.duo_oracle_e4m3_quantize.argtypes = [P, i64, ctypes.c_float, P]
         _lib = lib
@@ -149,3 +152,19 @@ def e4m3_quantize(x, inv_scale: float) -> np.ndarray:
     out = np.zeros(xb.shape, dtype=np.uint8)
     _load().duo_oracle_e4m3_quantize(xb.ctypes.data, xb.size, float(inv_scale), out.ctypes.data)
     return out
+
+
+def attend_rows_e4m3(q, k_codes, v_codes, k_scale: float, v_scale: float, scale: float):
+    """attend_rows over key/value rows [n, D] stored as E4M3 codes with per-head scales."""
+    lib = _load()
+    qb = _bits(q)
+    kc = np.ascontiguousarray(k_codes, dtype=np.uint8)
+    vc = np.ascontiguousarray(v_codes, dtype=np.uint8)
+    n, D = kc.shape
+    out = np.zeros(D, dtype=np.float64)
+    ws = np.zeros(1, dtype=np.float64)
+    rc = lib.duo_oracle_attend_rows_e4m3(qb.ctypes.data, kc.ctypes.data, vc.ctypes.data, n, D, float(k_scale),
+                                         float(v_scale), float(scale), out.ctypes.data, ws.ctypes.data)
+    if rc != 0:
+        raise ValueError("empty key list")
+    return out, float(ws[0])

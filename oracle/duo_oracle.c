@@ -241,3 +241,37 @@ void duo_oracle_e4m3_quantize(const uint16_t* x, int64_t n, float inv_scale, uin
         out[i] = duo_oracle_e4m3_code((double)prod);
     }
 }
+
+/* Attention of one query row (bf16) over n key/value rows held as E4M3 codes
+ * of a quantized retrieval cache: key element = value(code) * k_scale, value
+ * element = value(code) * v_scale; otherwise the same definition as
+ * duo_oracle_attend_rows. */
+int duo_oracle_attend_rows_e4m3(const uint16_t* q, const uint8_t* k_codes, const uint8_t* v_codes, int64_t n, int D,
+                                double k_scale, double v_scale, double scale, double* out, double* wsum) {
+    if (n <= 0) return -1;
+    double* s = (double*)malloc(sizeof(double) * (size_t)n);
+    if (!s) return -1;
+    double m = -INFINITY;
+    for (int64_t i = 0; i < n; ++i) {
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d)
+            dot += bf16_to_double(q[d]) * (duo_oracle_e4m3_value(k_codes[i * D + d]) * k_scale);
+        s[i] = scale * dot;
+        if (s[i] > m) m = s[i];
+    }
+    double denom = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        s[i] = exp(s[i] - m);
+        denom += s[i];
+    }
+    for (int d = 0; d < D; ++d) out[d] = 0.0;
+    double total = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        const double a = s[i] / denom;
+        total += a;
+        for (int d = 0; d < D; ++d) out[d] += a * (duo_oracle_e4m3_value(v_codes[i * D + d]) * v_scale);
+    }
+    if (wsum) *wsum = total;
+    free(s);
+    return 0;
+}

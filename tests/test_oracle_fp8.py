@@ -73,3 +73,36 @@ def test_quantize_is_fp32_product_then_nearest_code():
         # half a unit in the last place: 2^-4 relative for normals, 2^-10 absolute (scaled) below
         assert np.all(np.abs(back - xs)[normal] <= 2.0 ** -4 * np.abs(xs)[normal] * (1 + 1e-6))
         assert np.all(np.abs(back - xs)[a < 2.0 ** -6] <= 2.0 ** -10 / np.float32(inv) * (1 + 1e-6))
+
+
+def _grid_rows(g, n, D, lo=-2.0, hi=2.0):
+    """Random rows whose values are E4M3 codes in [lo, hi] (exact in bf16 too)."""
+    codes = [c for c in FINITE if lo <= oracle.e4m3_value(c) <= hi]
+    idx = torch.randint(0, len(codes), (n, D), generator=g)
+    c = np.array(codes, dtype=np.uint8)[idx.numpy()]
+    vals = np.vectorize(oracle.e4m3_value)(c)
+    return c, torch.tensor(vals, dtype=torch.float64).to(torch.bfloat16)
+
+
+def test_fp8_rows_equal_bf16_rows_when_values_are_exact():
+    g = torch.Generator().manual_seed(2)
+    D, n = 64, 37
+    kc, kb = _grid_rows(g, n, D)
+    vc, vb = _grid_rows(g, n, D)
+    q = torch.randn(D, generator=g).to(torch.bfloat16)
+    for ks, vs in ((1.0, 1.0), (0.25, 8.0)):  # powers of two scale exactly
+        got, wsum = oracle.attend_rows_e4m3(q, kc, vc, ks, vs, 0.125)
+        ref, _ = oracle.attend_rows(q, (kb.double() * ks).to(torch.bfloat16), (vb.double() * vs).to(torch.bfloat16),
+                                    0.125)
+        assert np.array_equal(got, ref)
+        assert abs(wsum - 1.0) < 1e-12
+
+
+def test_fp8_rows_constant_value_rows_return_that_value():
+    g = torch.Generator().manual_seed(3)
+    D, n = 32, 50
+    kc, _ = _grid_rows(g, n, D)
+    vc = np.full((n, D), oracle.e4m3_code(0.75), dtype=np.uint8)
+    q = torch.randn(D, generator=g).to(torch.bfloat16)
+    got, _ = oracle.attend_rows_e4m3(q, kc, vc, 1.7, 3.0, 0.2)
+    assert np.allclose(got, 0.75 * 3.0, rtol=0, atol=1e-12)
