@@ -11,7 +11,12 @@ tokens, all ranks), inputs resident in HBM. Sub-metrics: prefill TFLOP/s over
 unmasked positions, decode KV-read GB/s and tokens/s. `e2e` repeats the step
 through the same C ABI from pinned host buffers with the copies timed.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+At N = 1 the line also carries `secondary`: every other configuration of the
+benchmark definition (Llama-3-8B-shaped GQA decode at 128K, the MHA
+retrieval-ratio sweep of decode and chunked prefill at 64K, the 32-layer GQA
+stack at 1M), each with its own device time, roofline fraction and clock record.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-secondary]
 
 Under torchrun (N > 1) every rank runs an independent replica (the method has
 no cross-GPU exchange); the step time is the max over ranks.
@@ -88,12 +93,14 @@ def prefill_flops(w, mask, p0: int, n: int) -> float:
     return tot * 4.0 * w.head_dim * w.batch
 
 
-def decode_bytes(w, mask, L: int) -> float:
+def decode_bytes(w, mask, L: int, retr_elem: int = 2) -> float:
     """Bytes one decode step at cache length L must move: every visible K/V row once
-    (the new token's from the input), the new token's write, q and out."""
+    (the new token's from the input), the new token's write, q and out. Retrieval
+    rows take retr_elem bytes per element (2: bf16, 1: E4M3 codes)."""
     D, B = w.head_dim, w.batch
-    rows = sum((L + 1) if mask[g] else min(L + 1, w.sink + w.recent) for g in range(w.num_kv_heads))
-    return B * (rows * 2 * D * 2 + w.num_kv_heads * 2 * D * 2 + 2 * w.num_q_heads * D * 2)
+    retr = sum(L + 1 for g in range(w.num_kv_heads) if mask[g])
+    strm = sum(min(L + 1, w.sink + w.recent) for g in range(w.num_kv_heads) if not mask[g])
+    return B * ((retr * retr_elem + strm * 2) * 2 * D + w.num_kv_heads * 2 * D * 2 + 2 * w.num_q_heads * D * 2)
 
 
 def append_bytes(w, mask, L: int, n: int) -> float:
@@ -301,7 +308,8 @@ def run_gpu(args):
     append_gbs = sum(ab) / (t_ap * 1e-3) / 1e9
     decode_tok_s = w.batch * w.decode_steps / (t_dc * 1e-3)
     kernels = {
-        "prefill": {"bound": "tensor", "achieved": prefill_tflops, "peak": peaks["bf16_tflops_sustained"],
+        # Every prefill launch is timed on its own (CUDA events around it): the burst peak applies.
+        "prefill": {"bound": "tensor", "achieved": prefill_tflops, "peak": peaks["bf16_tflops"],
                     "unit": "TFLOP/s", "ms_per_step": t_pf, "launches_per_step": step.n_chunks},
         "decode": {"bound": "hbm", "achieved": decode_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                    "ms_per_step": t_dc, "launches_per_step": w.decode_steps},
@@ -319,6 +327,12 @@ def run_gpu(args):
     cpu = None
     if rank == 0:
         cpu = cpu_baseline(step, budget_s=args.cpu_budget)
+    secondary = None
+    if world == 1 and not args.no_secondary:
+        step.cache.close()
+        del step.chunks, step.dec
+        torch.cuda.empty_cache()
+        secondary = run_secondary(duo, peaks)
     res = {
         "metric": METRIC, "value": world * tok_per_step / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -330,7 +344,6 @@ def run_gpu(args):
                    "seq_len": step.T, "global_batch": w.batch * world,
                    "parallelism": "replicas" if world > 1 else "single", "l2": "inputs larger than L2"},
         "prefill": {"unmasked_tflops": prefill_tflops, "ms": t_pf, "unmasked_flop": sum(pf),
-                    "frac_of_measured_sustained": prefill_tflops / peaks["bf16_tflops_sustained"],
                     "frac_of_measured_burst": prefill_tflops / peaks["bf16_tflops"],
                     "frac_of_nominal_2250": prefill_tflops / 2250.0},
         "decode": {"kv_read_gbs": decode_gbs, "tokens_per_s": decode_tok_s, "us_per_step": 1e3 * t_dc / w.decode_steps,
@@ -342,6 +355,8 @@ def run_gpu(args):
     }
     if cpu is not None:
         res["cpu_baseline"] = cpu
+    if secondary is not None:
+        res["secondary"] = secondary
     if rank == 0:
         print(json.dumps(res))
     step.cache.close()
@@ -567,6 +582,9 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- secondary workloads
+L2_BYTES = 126 * 2**20
+
+
 def _fill_cache(duo, cache, w, layer, L, block=1 << 16):
     for c0 in range(0, L, block):
         n = min(block, L - c0)
@@ -574,99 +592,182 @@ def _fill_cache(duo, cache, w, layer, L, block=1 << 16):
         cache.append(layer, kk, vv)
 
 
-def _time_decode_steps(duo, cache, w, layers, L, steps):
-    """Device time of `steps` decode steps (one launch per layer each), back to back."""
-    qkv = [workloads.tokens(w, l, L, steps, device="cuda") for l in layers]
-    ins = [[tuple(x[:, t].contiguous() for x in qkv[i]) for t in range(steps)] for i in range(len(layers))]
-    o = torch.empty_like(ins[0][0][0])
-    lib, sp = duo._lib, torch.cuda.current_stream().cuda_stream
-    res = []
-    for rep in range(2):  # the first pass warms up
+def _with_clocks(fn, min_reps=3, max_s=10.0):
+    """Run fn() as warm-up until nvidia-smi has sampled at least 3 clock readings
+    (at least min_reps times, at most max_s seconds), then once more as the timed
+    run. Returns (the timed run's result, clocks over warm-up and timed run)."""
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    t0 = time.perf_counter()
+    reps = 0
+    while reps < min_reps or (clocks.samples() < 3 and time.perf_counter() - t0 < max_s):
+        fn()
+        reps += 1
+    res = fn()
+    clk = clocks.stop()
+    return res, dict(clk, window="warm-up through timed run", warmup_reps=reps)
+
+
+class DecodeCase:
+    """Decode steps of one workload (one launch per layer per step) on an
+    append-filled cache; device time per step with CUDA events."""
+
+    def __init__(self, duo, w, layers, steps, kv_format=0):
+        self.duo, self.w, self.layers, self.steps = duo, w, layers, steps
+        self.kv_format = kv_format
+        self.L = L = w.context
+        self.masks = [workloads.retrieval_mask(w, l) for l in range(w.num_layers)]
+        self.cache = duo.DuoCache(w.num_layers, w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.sink,
+                                  w.recent, L + steps + 1, [m for ms in self.masks for m in ms], kv_format=kv_format)
         for l in layers:
-            cache.set_length(l, L)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for t in range(steps):
-            for i, l in enumerate(layers):
-                q, k, v = ins[i][t]
-                if lib.duo_decode(cache.handle, l, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), sp):
+            _fill_cache(duo, self.cache, w, l, L)
+        qkv = [workloads.tokens(w, l, L, steps, device="cuda") for l in layers]
+        self.ins = [[tuple(x[:, t].contiguous() for x in qkv[i]) for t in range(steps)] for i in range(len(layers))]
+        self.out = torch.empty_like(self.ins[0][0][0])
+        elem = 1 if kv_format == duo.DUO_KV_E4M3 else 2
+        self.bytes_per_step = sum(statistics.fmean(decode_bytes(w, self.masks[l], L + s, elem) for s in range(steps))
+                                  for l in layers)
+        # A step whose reads fit in L2 would be served from L2 on the next step:
+        # flush L2 between timed steps then (a real model runs its other layers in between).
+        self.flush = (torch.empty(4 * L2_BYTES, dtype=torch.uint8, device="cuda")
+                      if self.bytes_per_step < 2 * L2_BYTES else None)
+
+    def run(self):
+        lib, sp = self.duo._lib, torch.cuda.current_stream().cuda_stream
+        for l in self.layers:
+            self.cache.set_length(l, self.L)
+        ev = []
+        if self.flush is None:
+            ev.append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+            ev[0][0].record()
+        for t in range(self.steps):
+            if self.flush is not None:
+                self.flush.fill_(t & 0xFF)
+                ev.append((torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)))
+                ev[-1][0].record()
+            for i, l in enumerate(self.layers):
+                q, k, v = self.ins[i][t]
+                if lib.duo_decode(self.cache.handle, l, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                  self.out.data_ptr(), sp):
                     raise RuntimeError("decode failed")
-        e1.record()
+            if self.flush is not None:
+                ev[-1][1].record()
+        if self.flush is None:
+            ev[0][1].record()
         torch.cuda.synchronize()
-        res.append(e0.elapsed_time(e1) * 1e-3 / steps)
-    if cache.error_flags():
-        raise RuntimeError("device error flag set")
-    return res[-1]
+        return sum(a.elapsed_time(b) for a, b in ev) * 1e-3 / self.steps
+
+    def result(self, peaks):
+        t, clk = _with_clocks(self.run)
+        if self.cache.error_flags():
+            raise RuntimeError("device error flag set")
+        w, gbs = self.w, self.bytes_per_step / t / 1e9
+        return {"workload": w.name + ("_e4m3" if self.kv_format else ""), "phase": "decode",
+                "retrieval_kv_format": "e4m3" if self.kv_format else "bf16",
+                "batch": w.batch, "context": self.L, "layers": len(self.layers),
+                "retrieval_kv_heads_per_layer": int(sum(self.masks[self.layers[0]])),
+                "steps": self.steps, "us_per_step": t * 1e6, "tokens_per_s": w.batch / t, "kv_read_gbs": gbs,
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / peaks["hbm_gbs"], "peak_source": peaks["source"]},
+                "frac_of_nominal_8000": gbs / 8000.0,
+                "l2": "flushed between steps" if self.flush is not None else "per-step reads larger than L2",
+                "clocks": clk}
+
+    def close(self):
+        self.cache.close()
+        del self.cache, self.ins, self.flush
+
+
+class PrefillCase:
+    """Chunked prefill of one workload (duo_prefill + duo_cache_append per chunk);
+    device time of the prefill launches with CUDA events around each."""
+
+    def __init__(self, duo, w):
+        self.duo, self.w = duo, w
+        self.mask = workloads.retrieval_mask(w)
+        self.cache = duo.DuoCache(1, w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.sink, w.recent,
+                                  w.prefill_len, self.mask)
+        q, k, v = workloads.tokens(w, 0, 0, w.prefill_len, device="cuda")
+        self.chunks = [(p0, tuple(x[:, p0:p0 + w.chunk].contiguous() for x in (q, k, v)))
+                       for p0 in range(0, w.prefill_len, w.chunk)]
+        self.out = torch.empty_like(self.chunks[0][1][0])
+        self.flop = sum(prefill_flops(w, self.mask, p0, w.chunk) for p0, _ in self.chunks)
+
+    def run(self):
+        self.cache.set_length(0, 0)
+        ev = []
+        for p0, (qc, kc, vc) in self.chunks:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            self.cache.prefill(0, qc, kc, vc, self.out)
+            e1.record()
+            ev.append((e0, e1))
+            self.cache.append(0, kc, vc)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) * 1e-3
+
+    def result(self, peaks):
+        t, clk = _with_clocks(self.run)
+        if self.cache.error_flags():
+            raise RuntimeError("device error flag set")
+        w, tf = self.w, self.flop / t / 1e12
+        return {"workload": w.name, "phase": "prefill", "batch": w.batch, "context": w.prefill_len, "chunk": w.chunk,
+                "retrieval_kv_heads": int(sum(self.mask)), "ms_prefill_kernels": t * 1e3, "unmasked_tflops": tf,
+                "unmasked_flop": self.flop,
+                "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": tf / peaks["bf16_tflops"], "peak_source": peaks["source"]},
+                "frac_of_nominal_2250": tf / 2250.0, "l2": "inputs larger than L2", "clocks": clk}
+
+    def close(self):
+        self.cache.close()
+        del self.cache, self.chunks
+
+
+def secondary_cases():
+    """(kind, workload, layers, steps) of every other configuration of the benchmark
+    definition: GQA decode at 128K, the MHA retrieval-ratio sweep (decode and
+    chunked prefill, recent 256 and 1024) and the 32-layer GQA stack at 1M; the
+    two GQA decodes also with E4M3 retrieval caches (the quantized cache the
+    pages' longest contexts rely on)."""
+    cases = [("decode", workloads.LLAMA3_GQA, [0], 20), ("decode_e4m3", workloads.LLAMA3_GQA, [0], 20)]
+    for ratio in (0.0, 0.25, 0.5, 0.75, 1.0):
+        cases.append(("decode", workloads.mha_sweep(ratio, recent=256), [0], 10))
+    for ratio in (0.0, 0.25):
+        cases.append(("decode", workloads.mha_sweep(ratio, recent=1024), [0], 10))
+    cases.append(("decode", workloads.GQA_STACK_1M, list(range(workloads.GQA_STACK_1M.num_layers)), 4))
+    cases.append(("decode_e4m3", workloads.GQA_STACK_1M, list(range(workloads.GQA_STACK_1M.num_layers)), 4))
+    for ratio in (0.0, 0.25, 0.5, 0.75, 1.0):
+        cases.append(("prefill", workloads.mha_sweep(ratio, recent=256, prefill=True), None, None))
+    cases.append(("prefill", workloads.mha_sweep(0.0, recent=1024, prefill=True), None, None))
+    return cases
+
+
+def run_secondary(duo, peaks, emit=None):
+    out = []
+    for kind, w, layers, steps in secondary_cases():
+        if kind == "prefill":
+            case = PrefillCase(duo, w)
+        else:
+            case = DecodeCase(duo, w, layers, steps, duo.DUO_KV_E4M3 if kind == "decode_e4m3" else duo.DUO_KV_BF16)
+        try:
+            r = case.result(peaks)
+        finally:
+            case.close()
+            torch.cuda.empty_cache()
+        out.append(r)
+        if emit is not None:
+            emit(r)
+    return out
 
 
 def run_sweep(args):
-    """The other workloads of the benchmark definition (decode at 128K and 1M,
-    the MHA retrieval-ratio sweep): one JSON line each, device time only."""
+    """The other workloads of the benchmark definition, one JSON line each
+    (device time, clocks sampled per line)."""
     torch.cuda.set_device(0)
     import __graft_entry__
     __graft_entry__.build()
     import mixed_head_kv_b200 as duo
-    peaks = load_peaks()
-    hbm = peaks["hbm_gbs"]
-    out = []
-
-    def emit(d):
-        print(json.dumps(d), flush=True)
-        out.append(d)
-
-    def decode_case(w, layers, steps):
-        L = w.context
-        masks = [workloads.retrieval_mask(w, l) for l in range(w.num_layers)]
-        cache = duo.DuoCache(w.num_layers, w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.sink, w.recent,
-                             L + steps + 1, [m for ms in masks for m in ms])
-        for l in layers:
-            _fill_cache(duo, cache, w, l, L)
-        t = _time_decode_steps(duo, cache, w, layers, L, steps)
-        byt = sum(statistics.fmean(decode_bytes(w, masks[l], L + s) for s in range(steps)) for l in layers)
-        emit({"workload": w.name, "phase": "decode", "batch": w.batch, "context": L, "layers": len(layers),
-              "us_per_step": t * 1e6, "tokens_per_s": w.batch / t, "kv_read_gbs": byt / t / 1e9,
-              "frac_of_measured_hbm": byt / t / 1e9 / hbm})
-        del cache
-        torch.cuda.empty_cache()
-
-    decode_case(workloads.LLAMA3_GQA, [0], 20)
-    for recent in (256, 1024):
-        for ratio in (0.0, 0.25, 0.5, 0.75, 1.0):
-            if recent == 1024 and ratio not in (0.0, 0.25):
-                continue
-            decode_case(workloads.mha_sweep(ratio, recent=recent), [0], 10)
-    decode_case(workloads.GQA_STACK_1M, list(range(workloads.GQA_STACK_1M.num_layers)), 4)
-
-    for recent, ratios in ((256, (0.0, 0.25, 0.5, 0.75, 1.0)), (1024, (0.0,))):
-        for ratio in ratios:
-            w = workloads.mha_sweep(ratio, recent=recent, prefill=True)
-            mask = workloads.retrieval_mask(w)
-            cache = duo.DuoCache(1, 1, 32, 32, 128, w.sink, w.recent, w.prefill_len, mask)
-            q, k, v = workloads.tokens(w, 0, 0, w.prefill_len, device="cuda")
-            chunks = [(p0, tuple(x[:, p0:p0 + w.chunk].contiguous() for x in (q, k, v)))
-                      for p0 in range(0, w.prefill_len, w.chunk)]
-            o = torch.empty_like(chunks[0][1][0])
-            times = []
-            for rep in range(2):
-                cache.set_length(0, 0)
-                ev = []
-                for p0, (qc, kc, vc) in chunks:
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0.record()
-                    cache.prefill(0, qc, kc, vc, o)
-                    e1.record()
-                    ev.append((e0, e1))
-                    cache.append(0, kc, vc)
-                torch.cuda.synchronize()
-                times.append(sum(a.elapsed_time(b) for a, b in ev) * 1e-3)
-            flop = sum(prefill_flops(w, mask, p0, w.chunk) for p0, _ in chunks)
-            emit({"workload": w.name, "phase": "prefill", "batch": 1, "context": w.prefill_len, "chunk": w.chunk,
-                  "ms_prefill_kernels": times[-1] * 1e3, "unmasked_tflops": flop / times[-1] / 1e12,
-                  "frac_of_measured_sustained": flop / times[-1] / 1e12 / peaks["bf16_tflops_sustained"]})
-            del cache, q, k, v, chunks
-            torch.cuda.empty_cache()
-    return out
+    return run_secondary(duo, load_peaks(), emit=lambda d: print(json.dumps(d), flush=True))
 
 
 # ----------------------------------------------------------------------------- memory footprint
@@ -713,7 +814,9 @@ def main(argv=None):
     ap.add_argument("--impl", default="duo", choices=["duo", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--sweep", action="store_true",
-                    help="time the other workloads (GQA decode at 128K and 1M, MHA ratio sweep) instead")
+                    help="time only the other workloads (GQA decode at 128K and 1M, MHA ratio sweep), a line each")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="leave the other workloads out of the main line (they run by default at N=1)")
     ap.add_argument("--memory", action="store_true",
                     help="print the KV-cache footprint of full attention against the mixed-head cache (no GPU)")
     args = ap.parse_args(argv)

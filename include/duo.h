@@ -25,7 +25,7 @@
  *  - Argument errors are reported before any launch and leave the cache
  *    unchanged. DUO_ERR_CUDA reports a failed launch or CUDA call.
  *  - Positions are absolute token indices within a sequence, starting at 0.
- *    All sequences of a batch have the same length.
+ *    Each sequence of a batch has its own cache length (duo_cache_seq_lens).
  *  - Positional encodings are the caller's: q and k arrive already encoded and
  *    cached tokens keep their original positions (no re-indexing).
  *  - Softmax scale: layout.softmax_scale, or 1/sqrt(head_dim) when it is 0.
@@ -113,7 +113,11 @@ typedef struct duo_cache duo_cache;
  *   streaming K, V pools  [n_streaming_heads_all_layers][batch][sink+recent][head_dim]
  *   streaming slot rule   position p < sink -> slot p; otherwise slot
  *                         sink + (p - sink) mod recent (fixed sinks + a ring)
- *   decode scratch        split-KV partial results, counters, an error word
+ *   decode scratch        split-KV partial results: batch x R x 256 splits x
+ *                         (num_q_heads / num_kv_heads) x (head_dim + 1) fp32,
+ *                         R = the most retrieval KV heads of any one layer
+ *                         (streaming heads write none); per-(sequence, KV head)
+ *                         split counters; an error word
  * The caller keeps ownership of dev_buf and frees it after duo_cache_free. */
 DUO_API duo_status duo_cache_alloc(const duo_layout* layout, const uint8_t* is_retrieval, void* dev_buf,
                            size_t buf_bytes, size_t* required_bytes, void* stream, duo_cache** out);
@@ -238,6 +242,8 @@ DUO_API duo_status duo_cache_error(duo_cache* cache, void* stream, uint32_t* fla
  *     whose kernels overlap on the GPU race on it: issue them on one stream.
  *   - The first call on a device looks up the array's address
  *     (cudaGetSymbolAddress, device current): make it before any stream capture.
+ *     The address is kept per device and context; after a device reset the
+ *     first call in the new context looks it up again (also before any capture).
  *   - DUO_ERR_SCRATCH_LIMIT when even one split per (sequence, retrieval head)
  *     does not fit: batch * retrieval KV heads * G * (head_dim + 1) * 4 bytes
  *     plus batch * num_kv_heads * 4 bytes of counters must stay below the limit.

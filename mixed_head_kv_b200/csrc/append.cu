@@ -2,74 +2,98 @@
 // cache for retrieval heads, a constant-length sink + recent cache for
 // streaming heads).
 //
-// One thread moves 16 bytes (8 bf16) of one K row and the same 16 bytes of the
-// V row. Reads walk the [B][n][Hkv][D] input in order (fully coalesced);
-// writes land in whole 16-byte pieces of 256-byte head rows. Streaming heads
-// skip the non-sink positions that a later position of the same call would
-// overwrite, so every destination slot is written at most once per call.
+// One CTA per (sequence b, appended token c): the token's K and V rows of all
+// KV heads are contiguous in the [B][n][Hkv][D] input, so the CTA reads them
+// coalesced and writes whole 16-byte pieces of each head's cache row. The slot
+// rules are evaluated once per token (uniform over the CTA):
+//   retrieval head: slot = position;
+//   streaming head: sink slot p < sink, else ring slot sink + (p - sink) mod
+//     recent, but only for the last `recent` positions of the call (earlier
+//     ring positions would be overwritten within the same call, so they are
+//     neither read nor written).
+// The threads walk the token's active heads (retrieval heads first, then the
+// streaming heads when the token is kept by them), 16 bytes of K and V per
+// thread and head, with up to four heads' loads in flight before their stores.
 // HBM-bound: bytes = 2 (K,V) x rows written x D x 2 B, read and written.
 #include "duo_internal.cuh"
 #include "sm100.cuh"
 
 namespace duo {
 
-__global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
-    grid_dependency_wait();  // launched with programmatic stream serialization
-    grid_launch_dependents();
-    const int vec_per_row = p.D / 8;
-    const int64_t total = static_cast<int64_t>(p.B) * p.n * p.Hkv * vec_per_row;
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int e = static_cast<int>(i % vec_per_row);
-        int64_t r = i / vec_per_row;
-        const int g = static_cast<int>(r % p.Hkv);
-        r /= p.Hkv;
-        const int64_t c = r % p.n;
-        const int b = static_cast<int>(r / p.n);
-        // Sequence b appends rows [0, n_b) at its own length (ragged batches).
-        const int64_t len_b = p.ragged ? p.seq_len[b] : p.len;
-        const int64_t n_b = p.ragged ? p.seq_n[b] : p.n;
-        if (c >= n_b) continue;
-        const int64_t pos = len_b + c;
-        const int64_t first_kept = len_b + n_b - p.R;  // ring positions below this are overwritten in-call
-        const int pool = p.heads.pool_idx[g];
-        bf16* dk;
-        bf16* dv;
-        int64_t off;
-        if (p.heads.is_retr[g]) {
-            off = ((static_cast<int64_t>(pool) * p.B + b) * p.max_len + pos) * p.D + e * 8;
-            dk = p.pools.rk;
-            dv = p.pools.rv;
-        } else {
-            int64_t slot;
-            if (pos < p.S) {
-                slot = pos;
-            } else if (pos >= first_kept) {
-                slot = p.S + (pos - p.S) % p.R;
-            } else {
-                continue;
+namespace {
+
+constexpr int kAppendThreads = 128;
+constexpr int kAppendUnroll = 4;
+
+// Token c of sequence b, at position pos; `end` = the sequence's length after the call.
+template <int D>
+__device__ __forceinline__ void append_token(const AppendParams& p, int b, int64_t c, int64_t pos, int64_t end) {
+    constexpr int LPR = D / 8;  // threads per row (16 bytes each)
+    constexpr int kHeadsPerPass = kAppendThreads / LPR;
+    int64_t sslot = -1;  // streaming slot, or -1 when the call itself evicts this position again
+    if (pos < p.S) sslot = pos;
+    else if (pos >= end - p.R) sslot = p.S + (pos - p.S) % p.R;
+    const int n_active = sslot >= 0 ? p.Hkv : p.n_retr;
+    const int e = threadIdx.x % LPR;
+    const int64_t row0 = (static_cast<int64_t>(b) * p.n + c) * p.Hkv;  // input row of head 0
+    for (int i0 = threadIdx.x / LPR; i0 < n_active; i0 += kAppendUnroll * kHeadsPerPass) {
+        uint4 kx[kAppendUnroll], vx[kAppendUnroll];
+        bf16* dk[kAppendUnroll];
+        bf16* dv[kAppendUnroll];
+#pragma unroll
+        for (int u = 0; u < kAppendUnroll; ++u) {
+            const int i = i0 + u * kHeadsPerPass;
+            dk[u] = nullptr;
+            dv[u] = nullptr;
+            if (i < n_active) {
+                const int g = p.order[i];
+                const int64_t pool = p.heads.pool_idx[g];
+                if (i < p.n_retr) {
+                    const int64_t off = ((pool * p.B + b) * p.max_len + pos) * D + e * 8;
+                    dk[u] = p.pools.rk + off;
+                    dv[u] = p.pools.rv + off;
+                } else {
+                    const int64_t off = ((pool * p.B + b) * p.W + sslot) * D + e * 8;
+                    dk[u] = p.pools.sk + off;
+                    dv[u] = p.pools.sv + off;
+                }
+                const int64_t src = (row0 + g) * D + e * 8;
+                kx[u] = ld_nc_v4(p.k + src);
+                vx[u] = ld_nc_v4(p.v + src);
             }
-            off = ((static_cast<int64_t>(pool) * p.B + b) * p.W + slot) * p.D + e * 8;
-            dk = p.pools.sk;
-            dv = p.pools.sv;
         }
-        const int64_t src = i * 8;  // input is [B][n][Hkv][D]: thread i owns elements [8i, 8i+8)
-        const uint4 kx = ld_nc_v4(p.k + src);
-        const uint4 vx = ld_nc_v4(p.v + src);
-        *reinterpret_cast<uint4*>(dk + off) = kx;
-        *reinterpret_cast<uint4*>(dv + off) = vx;
+#pragma unroll
+        for (int u = 0; u < kAppendUnroll; ++u) {
+            if (dk[u] != nullptr) {
+                *reinterpret_cast<uint4*>(dk[u]) = kx[u];
+                *reinterpret_cast<uint4*>(dv[u]) = vx[u];
+            }
+        }
     }
 }
 
+template <int D>
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(const AppendParams p) {
+    grid_dependency_wait();  // launched with programmatic stream serialization
+    grid_launch_dependents();
+    const int64_t c = blockIdx.x;
+    for (int b = blockIdx.y; b < p.B; b += gridDim.y) {
+        // Sequence b appends rows [0, n_b) at its own length (ragged batches).
+        const int64_t len_b = p.ragged ? p.seq_len[b] : p.len;
+        const int64_t n_b = p.ragged ? p.seq_n[b] : p.n;
+        if (c < n_b) append_token<D>(p, b, c, len_b + c, len_b + n_b);
+    }
+}
+
+}  // namespace
+
 cudaError_t launch_append(const AppendParams& p, cudaStream_t s) {
-    const int64_t total = static_cast<int64_t>(p.B) * p.n * p.Hkv * (p.D / 8);
-    if (total == 0) return cudaSuccess;
-    const int sms = p.num_sms > 0 ? p.num_sms : 148;
-    const int threads = 256;
-    int64_t blocks = (total + threads - 1) / threads;
-    const int64_t cap = static_cast<int64_t>(sms) * 8;  // grid-stride beyond 8 resident CTAs per SM
-    if (blocks > cap) blocks = cap;
-    return launch_pdl(append_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, s, p);
+    if (p.B <= 0 || p.n <= 0 || p.Hkv <= 0) return cudaSuccess;
+    if (p.n > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const dim3 grid(static_cast<unsigned>(p.n), static_cast<unsigned>(p.B < 65535 ? p.B : 65535));
+    if (p.D == 128) return launch_pdl(append_kernel<128>, grid, dim3(kAppendThreads), 0, s, p);
+    if (p.D == 64) return launch_pdl(append_kernel<64>, grid, dim3(kAppendThreads), 0, s, p);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace duo

@@ -19,7 +19,9 @@
 //    threads) race on the array: order them on one stream;
 //  - the first call on a device looks up the array's device address with
 //    cudaGetSymbolAddress (with that device current); make that first call
-//    before any stream capture.
+//    before any stream capture. The address is kept per device and context:
+//    after a device reset, the first call in the new context looks it up again
+//    (that call, too, belongs before any stream capture).
 #include <cstring>
 #include <mutex>
 
@@ -38,18 +40,44 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kStaticBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Device address of g_decode_scratch on the current device (looked up once per device).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// The driver's cuCtxGetCurrent, found through the runtime (the library links no driver stub).
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+// Device address of g_decode_scratch in the current context of device `dev`,
+// looked up once per (device, context): after a device reset the runtime makes
+// a new primary context in which the array is loaded again and may move, so a
+// changed context handle triggers a new lookup.
 cudaError_t scratch_address(int dev, void** out) {
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (get_ctx == nullptr) return cudaErrorNotSupported;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorInvalidDevice;
+    if (g_scratch_addr[dev] == nullptr || ctx == nullptr || g_scratch_ctx[dev] != ctx) {
         void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);  // makes the context current if needed
         if (e != cudaSuccess) return e;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorInvalidDevice;
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = ctx;
     }
     *out = g_scratch_addr[dev];
     return cudaSuccess;

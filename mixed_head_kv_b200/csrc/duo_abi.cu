@@ -23,14 +23,17 @@ struct Regions {
     size_t retr_pool, strm_pool, part_o, part_lse, counters, err, total;
 };
 
-Regions regions_for(const duo_layout& L, int64_t n_retr_all, int64_t n_strm_all) {
+// Split-KV partials are written by retrieval (b, KV head, split) items only, indexed
+// by the head's rank among the layer's retrieval heads: the scratch holds
+// batch x (most retrieval heads of any layer) x kDecodeMaxSplits partials.
+Regions regions_for(const duo_layout& L, int64_t n_retr_all, int64_t n_strm_all, int64_t max_retr_layer) {
     Regions r{};
     const size_t D = static_cast<size_t>(L.head_dim);
     const size_t W = static_cast<size_t>(L.sink) + static_cast<size_t>(L.recent);
     const size_t G = static_cast<size_t>(L.num_q_heads / L.num_kv_heads);
     r.retr_pool = align_up(static_cast<size_t>(n_retr_all) * L.batch * static_cast<size_t>(L.max_len) * D * 2);
     r.strm_pool = align_up(static_cast<size_t>(n_strm_all) * L.batch * W * D * 2);
-    const size_t items = static_cast<size_t>(L.batch) * L.num_kv_heads * kDecodeMaxSplits;
+    const size_t items = static_cast<size_t>(L.batch) * static_cast<size_t>(max_retr_layer) * kDecodeMaxSplits;
     r.part_o = align_up(items * G * D * sizeof(float));
     r.part_lse = align_up(items * G * sizeof(float));
     r.counters = align_up(static_cast<size_t>(L.batch) * L.num_kv_heads * sizeof(uint32_t));
@@ -156,9 +159,14 @@ duo_status duo_cache_alloc(const duo_layout* layout, const uint8_t* is_retrieval
     if (st != DUO_OK) return st;
     const duo_layout& L = *layout;
     const int64_t n = static_cast<int64_t>(L.num_layers) * L.num_kv_heads;
-    int64_t n_retr = 0;
-    for (int64_t i = 0; i < n; ++i) n_retr += is_retrieval[i];
-    const Regions reg = regions_for(L, n_retr, n - n_retr);
+    int64_t n_retr = 0, max_retr_layer = 0;
+    for (int32_t l = 0; l < L.num_layers; ++l) {
+        int64_t nl = 0;
+        for (int32_t g = 0; g < L.num_kv_heads; ++g) nl += is_retrieval[static_cast<int64_t>(l) * L.num_kv_heads + g];
+        n_retr += nl;
+        if (nl > max_retr_layer) max_retr_layer = nl;
+    }
+    const Regions reg = regions_for(L, n_retr, n - n_retr, max_retr_layer);
     if (required_bytes) *required_bytes = reg.total;
     if (!dev_buf) return DUO_OK;
     if (!out) return DUO_ERR_INVALID_ARG;
@@ -343,7 +351,6 @@ duo_status append_impl(duo_cache* c, int32_t layer, const void* k, const void* v
     p.S = c->lay.sink;
     p.R = c->lay.recent;
     p.W = c->W;
-    p.num_sms = c->num_sms;
     p.ragged = uniform ? 0 : 1;
     if (!uniform) {
         for (int32_t b = 0; b < B; ++b) {
@@ -352,6 +359,12 @@ duo_status append_impl(duo_cache* c, int32_t layer, const void* k, const void* v
         }
     }
     fill_heads(c, layer, &p.heads);
+    for (int pass = 0; pass < 2; ++pass) {
+        int n = pass == 0 ? 0 : p.n_retr;
+        for (int g = 0; g < p.Hkv; ++g)
+            if ((p.heads.is_retr[g] != 0) == (pass == 0)) p.order[n++] = static_cast<int16_t>(g);
+        if (pass == 0) p.n_retr = n;
+    }
     if (launch_append(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUO_ERR_CUDA;
     for (int32_t b = 0; b < B; ++b) L[b] += n_tok[b];
     return DUO_OK;

@@ -76,9 +76,10 @@ struct AppendParams {
     int64_t n;        // tokens appended (uniform batch); rows per sequence of k and v
     int64_t max_len;
     int32_t B, Hkv, D, S, R, W;
-    int32_t num_sms;
     int32_t ragged;   // 1: per-sequence seq_len / seq_n below
+    int32_t n_retr;   // retrieval KV heads of the layer, listed first in order[]
     HeadMap heads;
+    int16_t order[DUO_MAX_KV_HEADS];   // KV heads, retrieval heads first
     int64_t seq_len[kMaxRaggedBatch];  // tokens cached before this call, per sequence
     int64_t seq_n[kMaxRaggedBatch];    // tokens appended, per sequence (<= n)
 };

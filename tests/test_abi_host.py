@@ -50,7 +50,9 @@ def _expected_bytes(L, mask):
     nr = sum(mask)
     ns = len(mask) - nr
     D, B, W, G = L.head_dim, L.batch, L.sink + L.recent, L.num_q_heads // L.num_kv_heads
-    items = B * L.num_kv_heads * 256
+    H = L.num_kv_heads
+    max_retr = max(sum(mask[l * H:(l + 1) * H]) for l in range(L.num_layers))
+    items = B * max_retr * 256  # partials: retrieval heads only, per layer
     return (2 * a(nr * B * L.max_len * D * 2) + 2 * a(ns * B * W * D * 2) + a(items * G * D * 4)
             + a(items * G * 4) + a(B * L.num_kv_heads * 4) + a(4))
 
@@ -71,7 +73,8 @@ def test_memory_reduction_shape():
     _, mixed, _ = duo.duo_cache_alloc(L, [1] * 8 + [0] * 24)
     pools_full = 2 * 32 * 32768 * 128 * 2
     pools_mixed = 2 * (8 * 32768 + 24 * 320) * 128 * 2
-    assert full - mixed == pools_full - pools_mixed
+    scratch = lambda n_retr: n_retr * 256 * 128 * 4 + n_retr * 256 * 4  # split-KV partials of retrieval heads
+    assert full - mixed == pools_full - pools_mixed + scratch(32) - scratch(8)
 
 
 @pytest.mark.parametrize("bad", [
