@@ -57,6 +57,20 @@ typedef enum duo_status {
     DUO_ERR_SCRATCH_LIMIT = 7 /* the request needs more than DUO_STATIC_SCRATCH_BYTES */
 } duo_status;
 
+/* Storage format of the retrieval heads' caches (streaming caches are always
+ * bf16). The pages reach their longest contexts only with a quantized KV cache
+ * (DuoAttention abstract: 3.3 million tokens on one GPU "combined with
+ * quantization"); this library offers FP8 E4M3 with one scale per (layer, KV
+ * head) for K and one for V:
+ *   DUO_KV_BF16  bf16 rows (default)
+ *   DUO_KV_E4M3  each element is stored as the E4M3 code of x * inv_scale (the
+ *                product in fp32, inv_scale the fp32 reciprocal of the head's
+ *                scale), rounded to nearest with ties to even and saturated to
+ *                +-448, and read back as value(code) * scale. Halves the bytes a
+ *                decode step reads from retrieval caches. */
+#define DUO_KV_BF16 0
+#define DUO_KV_E4M3 1
+
 /* Largest head counts the kernels accept. */
 #define DUO_MAX_Q_HEADS 256
 #define DUO_MAX_KV_HEADS 128
@@ -77,6 +91,7 @@ typedef enum duo_status {
  *   recent        recent tokens kept by streaming heads (>= 1); includes the
  *                 query's own token, so a streaming query at position p attends
  *                 to { j <= p : j < sink or p - j < recent }
+ *   kv_format     DUO_KV_BF16 or DUO_KV_E4M3 (retrieval caches; see above)
  *   max_len       capacity of every retrieval cache in tokens
  *   softmax_scale 0 selects 1/sqrt(head_dim) */
 typedef struct duo_layout {
@@ -87,7 +102,7 @@ typedef struct duo_layout {
     int32_t head_dim;
     int32_t sink;
     int32_t recent;
-    int32_t reserved0;
+    int32_t kv_format; /* DUO_KV_BF16 or DUO_KV_E4M3: storage of the retrieval caches */
     int64_t max_len;
     float softmax_scale;
     int32_t reserved1;
@@ -110,6 +125,7 @@ typedef struct duo_cache duo_cache;
  *   out           out: the new cache object (when dev_buf != NULL)
  * Device layout inside dev_buf (offsets in required_bytes order):
  *   retrieval K, V pools  [n_retrieval_heads_all_layers][batch][max_len][head_dim]
+ *                         (bf16, or one-byte E4M3 codes for DUO_KV_E4M3)
  *   streaming K, V pools  [n_streaming_heads_all_layers][batch][sink+recent][head_dim]
  *   streaming slot rule   position p < sink -> slot p; otherwise slot
  *                         sink + (p - sink) mod recent (fixed sinks + a ring)
@@ -118,6 +134,9 @@ typedef struct duo_cache duo_cache;
  *                         R = the most retrieval KV heads of any one layer
  *                         (streaming heads write none); per-(sequence, KV head)
  *                         split counters; an error word
+ *   E4M3 scales           DUO_KV_E4M3 only: [num_layers][num_kv_heads] x 4 fp32
+ *                         (k_scale, v_scale and their fp32 reciprocals), 1 until
+ *                         duo_cache_set_kv_scales
  * The caller keeps ownership of dev_buf and frees it after duo_cache_free. */
 DUO_API duo_status duo_cache_alloc(const duo_layout* layout, const uint8_t* is_retrieval, void* dev_buf,
                            size_t buf_bytes, size_t* required_bytes, void* stream, duo_cache** out);
@@ -161,6 +180,9 @@ DUO_API duo_status duo_cache_append_ragged(duo_cache* cache, int32_t layer, cons
  * streaming heads over the sinks and the recent window, read from the
  * streaming cache for positions < len and from k/v for the chunk.
  * Does NOT modify the cache: call duo_cache_append(layer, k, v, n_tok) after it.
+ * DUO_KV_E4M3 caches: the tensor-core prefill reads bf16 tiles only, so a chunk
+ * is refused (DUO_ERR_STATE) once a retrieval head of the layer holds tokens;
+ * prefill the prompt in one chunk, then decode.
  * Each sequence's chunk starts at its own length len_b (a ragged batch needs
  * batch <= DUO_MAX_RAGGED_BATCH, else DUO_ERR_STATE).
  * DUO_ERR_CAPACITY if a retrieval head could not hold len_b + n_tok tokens. */
@@ -203,6 +225,16 @@ DUO_API duo_status duo_cache_len(const duo_cache* cache, int32_t layer, int64_t*
  * the caller's to restore). 0 <= len <= max_len. */
 DUO_API duo_status duo_cache_set_len(duo_cache* cache, int32_t layer, int64_t len);
 
+/* duo_cache_set_kv_scales — per-KV-head scales of a DUO_KV_E4M3 cache.
+ *   k_scale, v_scale  host [num_kv_heads], finite and > 0 (the entries of
+ *                     streaming heads are checked but not used)
+ * The scales apply to tokens appended (and decoded) afterwards: set them before
+ * the layer's first append. Copies them to the device on `stream`.
+ * DUO_ERR_STATE for a bf16 cache; DUO_ERR_INVALID_ARG for a bad scale (nothing
+ * changes). */
+DUO_API duo_status duo_cache_set_kv_scales(duo_cache* cache, int32_t layer, const float* k_scale,
+                                           const float* v_scale, void* stream);
+
 /* duo_cache_seq_lens — per-sequence lengths of `layer`.
  *   lens  host [batch], written (host values; no sync) */
 DUO_API duo_status duo_cache_seq_lens(const duo_cache* cache, int32_t layer, int64_t* lens);
@@ -213,6 +245,7 @@ DUO_API duo_status duo_cache_set_seq_lens(duo_cache* cache, int32_t layer, const
 
 /* duo_cache_views — where one KV head's cache lives, for inspection.
  *   k, v          out: device pointers to [batch][slots][head_dim] bf16
+ *                 (uint8 E4M3 codes for a retrieval head of a DUO_KV_E4M3 cache)
  *   slots         out: max_len (retrieval) or sink + recent (streaming)
  *   is_retrieval  out: 1 or 0
  * Any out pointer may be NULL. */
@@ -220,8 +253,9 @@ DUO_API duo_status duo_cache_views(const duo_cache* cache, int32_t layer, int32_
                            int64_t* slots, int32_t* is_retrieval);
 
 /* duo_cache_error — read and clear the device-side error word of the cache
- * (bit flags set by kernels whose bounded waits ran out). Synchronizes
- * `stream`. *flags = 0 when no kernel reported an error. */
+ * (bit flags set by kernels whose bounded waits ran out: DUO_ERR_BIT_PREFILL_WAIT,
+ * DUO_ERR_BIT_DECODE_COPY). Synchronizes `stream`. *flags = 0 when no kernel
+ * reported an error. */
 DUO_API duo_status duo_cache_error(duo_cache* cache, void* stream, uint32_t* flags);
 
 /* duo_decode_static_scratch — duo_decode for callers that cannot allocate device
@@ -252,6 +286,32 @@ DUO_API duo_status duo_cache_error(duo_cache* cache, void* stream, uint32_t* fla
 #define DUO_STATIC_SCRATCH_BYTES (16u * 1024u * 1024u)
 DUO_API duo_status duo_decode_static_scratch(duo_cache* cache, int32_t layer, const void* q, const void* k_new,
                                              const void* v_new, void* out, void* stream);
+
+/* duo_cache_test_wait_timeout — a test of the kernels' failure detection; not
+ * for production use. Every wait of a kernel on an asynchronous copy is bounded
+ * (1 s); when one runs out the kernel sets a bit in the cache's error word
+ * (duo_cache_error), finishes without the missing data and returns, and the
+ * call that launched it has already returned DUO_OK. This call arms the next
+ * launch of the kinds in `launches` on this cache to exercise that path without
+ * any fault: one of its CTAs does not issue one of its copies, and the wait for
+ * that copy gives up after `timeout_ns` (1 us .. 1 s) instead of 1 s. Every
+ * other copy is issued and waited for as usual, so nothing is left in flight.
+ *   DUO_TEST_WAIT_DECODE  the next duo_decode launch: warp 0 of its first CTA
+ *                         withholds its first K/V block; error bit
+ *                         DUO_ERR_BIT_DECODE_COPY; that step's output is wrong,
+ *                         the cache update and every later call are not affected
+ *   DUO_TEST_WAIT_PREFILL the next duo_prefill launch: its first CTA withholds
+ *                         its first K tile; the CTA's MMA issuer gives up, the
+ *                         CTA's other roles stop at their next wait and drain
+ *                         what they issued; error bit DUO_ERR_BIT_PREFILL_WAIT;
+ *                         the output rows of that CTA's work items are not
+ *                         written, every other item's rows are
+ * 0 disarms. DUO_ERR_INVALID_ARG for an unknown kind or a limit out of range. */
+#define DUO_TEST_WAIT_DECODE 1
+#define DUO_TEST_WAIT_PREFILL 2
+#define DUO_ERR_BIT_PREFILL_WAIT 1u  /* duo_cache_error bits */
+#define DUO_ERR_BIT_DECODE_COPY 2u
+DUO_API duo_status duo_cache_test_wait_timeout(duo_cache* cache, int32_t launches, uint64_t timeout_ns);
 
 /* duo_status_str — static description of a status code. */
 DUO_API const char* duo_status_str(duo_status status);

@@ -38,17 +38,24 @@ DUO_MAX_Q_HEADS = 256
 DUO_MAX_KV_HEADS = 128
 
 DUO_MAX_RAGGED_BATCH = 64  # sequences of different lengths per batch (include/duo.h)
+DUO_KV_BF16 = 0  # cache formats of the retrieval heads (include/duo.h)
+DUO_KV_E4M3 = 1
 
 EXPORTED = ("duo_cache_alloc", "duo_cache_free", "duo_cache_append", "duo_prefill", "duo_decode",
             "duo_cache_len", "duo_cache_set_len", "duo_cache_views", "duo_cache_error", "duo_status_str",
             "duo_decode_static_scratch", "duo_cache_append_ragged", "duo_cache_seq_lens",
-            "duo_cache_set_seq_lens", "duo_prefill_ragged")
+            "duo_cache_set_seq_lens", "duo_prefill_ragged", "duo_cache_set_kv_scales",
+            "duo_cache_test_wait_timeout")
+DUO_TEST_WAIT_DECODE = 1  # duo_cache_test_wait_timeout kinds and duo_cache_error bits (include/duo.h)
+DUO_TEST_WAIT_PREFILL = 2
+DUO_ERR_BIT_PREFILL_WAIT = 1
+DUO_ERR_BIT_DECODE_COPY = 2
 
 
 class duo_layout(ctypes.Structure):
     _fields_ = [("num_layers", ctypes.c_int32), ("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("sink", ctypes.c_int32),
-                ("recent", ctypes.c_int32), ("reserved0", ctypes.c_int32), ("max_len", ctypes.c_int64),
+                ("recent", ctypes.c_int32), ("kv_format", ctypes.c_int32), ("max_len", ctypes.c_int64),
                 ("softmax_scale", ctypes.c_float), ("reserved1", ctypes.c_int32)]
 
 
@@ -81,12 +88,16 @@ _lib.duo_cache_views.argtypes = [_P, _I32, _I32, ctypes.POINTER(_P), ctypes.POIN
                                  ctypes.POINTER(_I32)]
 _lib.duo_cache_append_ragged.restype = _ST
 _lib.duo_cache_append_ragged.argtypes = [_P, _I32, _P, _P, ctypes.POINTER(_I64), _I64, _P]
+_lib.duo_cache_set_kv_scales.restype = _ST
+_lib.duo_cache_set_kv_scales.argtypes = [_P, _I32, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_float), _P]
 _lib.duo_prefill_ragged.restype = _ST
 _lib.duo_prefill_ragged.argtypes = [_P, _I32, _P, _P, _P, _P, ctypes.POINTER(_I64), _I64, _P]
 _lib.duo_cache_seq_lens.restype = _ST
 _lib.duo_cache_seq_lens.argtypes = [_P, _I32, ctypes.POINTER(_I64)]
 _lib.duo_cache_set_seq_lens.restype = _ST
 _lib.duo_cache_set_seq_lens.argtypes = [_P, _I32, ctypes.POINTER(_I64)]
+_lib.duo_cache_test_wait_timeout.restype = _ST
+_lib.duo_cache_test_wait_timeout.argtypes = [_P, _I32, ctypes.c_uint64]
 _lib.duo_cache_error.restype = _ST
 _lib.duo_cache_error.argtypes = [_P, _P, ctypes.POINTER(ctypes.c_uint32)]
 
@@ -126,8 +137,8 @@ def duo_status_str(status: int) -> str:
 
 
 def make_layout(num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, recent, max_len,
-                softmax_scale=0.0) -> duo_layout:
-    return duo_layout(num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, recent, 0, max_len,
+                softmax_scale=0.0, kv_format=0) -> duo_layout:
+    return duo_layout(num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, recent, kv_format, max_len,
                       softmax_scale, 0)
 
 
@@ -195,6 +206,13 @@ def duo_prefill_ragged(handle, layer, q, k, v, out, n_tok: Sequence[int], max_to
                                    _stream(stream) if q is not None else None)
 
 
+def duo_cache_set_kv_scales(handle, layer, k_scale: Sequence[float], v_scale: Sequence[float], stream=None) -> int:
+    """Per-KV-head scales of an E4M3 cache (host lists [num_kv_heads])."""
+    k = (ctypes.c_float * max(1, len(k_scale)))(*[float(x) for x in k_scale])
+    v = (ctypes.c_float * max(1, len(v_scale)))(*[float(x) for x in v_scale])
+    return _lib.duo_cache_set_kv_scales(handle, layer, k, v, _stream(stream))
+
+
 def duo_cache_seq_lens(handle, layer, batch: int):
     lens = (_I64 * batch)()
     st = _lib.duo_cache_seq_lens(handle, layer, lens)
@@ -213,6 +231,11 @@ def duo_cache_views(handle, layer, kv_head):
     return st, k.value, v.value, slots.value, r.value
 
 
+def duo_cache_test_wait_timeout(handle, launches: int, timeout_ns: int) -> int:
+    """Arm the next launch of the given kinds to test the bounded waits (include/duo.h)."""
+    return _lib.duo_cache_test_wait_timeout(handle, launches, timeout_ns)
+
+
 def duo_cache_error(handle, stream=None):
     f = ctypes.c_uint32(0)
     st = _lib.duo_cache_error(handle, _stream(stream), ctypes.byref(f))
@@ -223,10 +246,10 @@ class DuoCache:
     """A cache handle plus the torch uint8 buffer that backs it (owned here)."""
 
     def __init__(self, num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, recent, max_len,
-                 is_retrieval: Sequence[int], softmax_scale=0.0, device="cuda", stream=None):
+                 is_retrieval: Sequence[int], softmax_scale=0.0, device="cuda", stream=None, kv_format=0):
         import torch
         self.layout = make_layout(num_layers, batch, num_q_heads, num_kv_heads, head_dim, sink, recent, max_len,
-                                  softmax_scale)
+                                  softmax_scale, kv_format)
         self.is_retrieval = [int(x) for x in is_retrieval]
         st, req, _ = duo_cache_alloc(self.layout, self.is_retrieval)
         _check(st, "duo_cache_alloc(size)")
@@ -288,14 +311,20 @@ class DuoCache:
         return f
 
     def head_view(self, layer, kv_head):
-        """(k, v, is_retrieval): torch views [batch, slots, head_dim] of one KV head's cache."""
+        """(k, v, is_retrieval): torch views [batch, slots, head_dim] of one KV head's cache
+        (bf16, or uint8 E4M3 codes for the retrieval heads of an E4M3 cache)."""
         import torch
         st, kp, vp, slots, r = duo_cache_views(self.handle, layer, kv_head)
         _check(st, "duo_cache_views")
         B, D = self.layout.batch, self.layout.head_dim
-        n = B * slots * D * 2  # bytes
+        codes = bool(r) and self.layout.kv_format == DUO_KV_E4M3
+        n = B * slots * D * (1 if codes else 2)  # bytes
 
         def view(ptr):
             start = ptr - self.buffer.data_ptr()
-            return self.buffer[start:start + n].view(torch.bfloat16).view(B, slots, D)
+            raw = self.buffer[start:start + n]
+            return (raw if codes else raw.view(torch.bfloat16)).view(B, slots, D)
         return view(kp), view(vp), r
+
+    def set_kv_scales(self, layer, k_scale, v_scale, stream=None):
+        _check(duo_cache_set_kv_scales(self.handle, layer, k_scale, v_scale, stream), "duo_cache_set_kv_scales")

@@ -172,17 +172,167 @@ __device__ __forceinline__ void merge_lanes(DecState<G>& st, int off) {
     }
 }
 
+// Test of the bounded waits (DecodeParams::test_withhold): warp 0 of CTA 0 does
+// not issue its first copy, so its wait on it gives up after timeout_ns and the
+// CTA reports kErrDecodeCopy. Every other copy is issued and waited for as usual.
+struct WaitTest {
+    bool withhold;
+    uint64_t timeout_ns;
+};
+
+// Eight E4M3 codes (8 bytes) as four packed fp32 pairs.
+__device__ __forceinline__ void e4m3x8_to_f2(const uint2& c, uint64_t (&r)[4]) {
+    const uint32_t w[2] = {c.x, c.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        float a, b, d, e;
+        e4m3x2_to_f32(static_cast<uint16_t>(w[i] & 0xFFFFu), a, b);
+        e4m3x2_to_f32(static_cast<uint16_t>(w[i] >> 16), d, e);
+        r[2 * i] = f2pack(a, b);
+        r[2 * i + 1] = f2pack(d, e);
+    }
+}
+
+// accumulate() for rows held as E4M3 codes (an E4M3 retrieval cache): this
+// lane's 8 codes of K and V per row group. The head's scales are applied
+// outside (k_scale folded into q2, v_scale into the partial output).
+template <int D, int G, int U>
+__device__ __forceinline__ void accumulate8(DecState<G>& st, const uint64_t (&q2)[G][4], const uint2 (&kc)[U],
+                                            const uint2 (&vc)[U], const bool (&valid)[U]) {
+    constexpr int LPR = D / 8;
+    float s[U][G];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        uint64_t k2[4];
+        e4m3x8_to_f2(kc[u], k2);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            uint64_t acc = f2pack(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc = ffma2(q2[h][i], k2[i], acc);
+            float lo, hi;
+            f2unpack(acc, lo, hi);
+            s[u][h] = lo + hi;
+        }
+    }
+#pragma unroll
+    for (int off = LPR / 2; off >= 1; off >>= 1) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) s[u][h] += __shfl_xor_sync(0xffffffffu, s[u][h], off);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        if (!valid[u]) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) s[u][h] = -INFINITY;
+        }
+    }
+    uint64_t v2[U][4];
+#pragma unroll
+    for (int u = 0; u < U; ++u) e4m3x8_to_f2(vc[u], v2[u]);
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        float mb = s[0][h];
+#pragma unroll
+        for (int u = 1; u < U; ++u) mb = fmaxf(mb, s[u][h]);
+        if (mb > st.m[h] + kDecodeRescale) {
+            const float f = fast_exp2(st.m[h] - mb);
+            st.m[h] = mb;
+            st.l[h] *= f;
+            const uint64_t f2 = f2pack(f, f);
+            const uint64_t z2 = f2pack(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) st.o[h][i] = ffma2(st.o[h][i], f2, z2);
+        }
+        if (st.m[h] == -INFINITY) continue;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const float pu = fast_exp2(s[u][h] - st.m[h]);
+            st.l[h] += pu;
+            const uint64_t p2 = f2pack(pu, pu);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) st.o[h][i] = ffma2(p2, v2[u][i], st.o[h][i]);
+        }
+    }
+}
+
+// warp_stream() for an E4M3 retrieval cache: rows of D one-byte codes, so a
+// 4 KB block holds twice the rows; a lane reads 8 codes (8 bytes) of a row.
+template <int D, int G>
+__device__ bool warp_stream8(DecState<G>& st, const uint64_t (&q2)[G][4], const uint8_t* kbase, const uint8_t* vbase,
+                             int64_t r0, int64_t r1, uint32_t ring, uint32_t bars, const WaitTest& wt) {
+    using Gm = Geom<D, G>;
+    constexpr int BLK8 = Gm::kBlockBytes / D;  // rows per block of codes
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % Gm::LPR;
+    const int rsub = lane / Gm::LPR;
+    const int64_t nblk = (r1 - r0 + BLK8 - 1) / BLK8;
+    auto issue = [&](int64_t i) {
+        if (i == 0 && wt.withhold) return;  // test of the bounded wait: this copy is never issued
+        const int stg = static_cast<int>(i % Gm::kStages);
+        const int64_t a = r0 + i * BLK8;
+        const int64_t n = (r1 - a < BLK8) ? (r1 - a) : BLK8;
+        const uint32_t bytes = static_cast<uint32_t>(n * D);
+        const uint32_t bar = bars + 8u * stg;
+        const uint32_t dst = ring + stg * Gm::kStageBytes;
+        mbar_arrive_expect_tx(bar, 2 * bytes);
+        bulk_load(dst, kbase + a * D, bytes, bar);
+        bulk_load(dst + Gm::kBlockBytes, vbase + a * D, bytes, bar);
+    };
+    if (lane == 0) {
+        for (int64_t i = 0; i < nblk && i < Gm::kStages; ++i) issue(i);
+    }
+    for (int64_t i = 0; i < nblk; ++i) {
+        const int stg = static_cast<int>(i % Gm::kStages);
+        if (!mbar_wait(bars + 8u * stg, static_cast<uint32_t>((i / Gm::kStages) & 1), nullptr,
+                       i == 0 && wt.withhold ? wt.timeout_ns : kWaitTimeoutNs)) {
+            for (int64_t j = i + 1; j < nblk && j < i + Gm::kStages; ++j)
+                mbar_wait(bars + 8u * static_cast<uint32_t>(j % Gm::kStages),
+                          static_cast<uint32_t>((j / Gm::kStages) & 1), nullptr);
+            return false;
+        }
+        const int64_t a = r0 + i * BLK8;
+        const int rows = static_cast<int>((r1 - a < BLK8) ? (r1 - a) : BLK8);
+        const uint32_t kst = ring + stg * Gm::kStageBytes;
+        const uint32_t vst = kst + Gm::kBlockBytes;
+#pragma unroll
+        for (int u0 = 0; u0 < BLK8 / Gm::RPW; u0 += kGroupRows) {
+            uint2 kc[kGroupRows], vc[kGroupRows];
+            bool valid[kGroupRows];
+#pragma unroll
+            for (int u = 0; u < kGroupRows; ++u) {
+                const int row = (u0 + u) * Gm::RPW + rsub;
+                valid[u] = row < rows;
+                const uint32_t off = static_cast<uint32_t>(row * D + sub * 8);
+                kc[u] = valid[u] ? lds64(kst + off) : make_uint2(0, 0);
+                vc[u] = valid[u] ? lds64(vst + off) : make_uint2(0, 0);
+            }
+            accumulate8<D, G, kGroupRows>(st, q2, kc, vc, valid);
+        }
+        __syncwarp();
+        if (lane == 0 && i + Gm::kStages < nblk) {
+            fence_proxy_async_smem();
+            issue(i + Gm::kStages);
+        }
+    }
+    return true;
+}
+
 // Stream rows [r0, r1) (except `skip`) of one head through this warp's ring.
 // Returns false if a copy did not complete within the wait limit.
 template <int D, int G>
 __device__ bool warp_stream(DecState<G>& st, const uint64_t (&q2)[G][4], const bf16* kbase, const bf16* vbase,
-                            int64_t r0, int64_t r1, int64_t skip, uint32_t ring, uint32_t bars) {
+                            int64_t r0, int64_t r1, int64_t skip, uint32_t ring, uint32_t bars, const WaitTest& wt) {
     using Gm = Geom<D, G>;
     const int lane = threadIdx.x & 31;
     const int sub = lane % Gm::LPR;
     const int rsub = lane / Gm::LPR;
     const int64_t nblk = (r1 - r0 + Gm::BLK - 1) / Gm::BLK;
     auto issue = [&](int64_t i) {
+        if (i == 0 && wt.withhold) return;  // test of the bounded wait: this copy is never issued
         const int stg = static_cast<int>(i % Gm::kStages);
         const int64_t a = r0 + i * Gm::BLK;
         const int64_t n = (r1 - a < Gm::BLK) ? (r1 - a) : Gm::BLK;
@@ -198,7 +348,8 @@ __device__ bool warp_stream(DecState<G>& st, const uint64_t (&q2)[G][4], const b
     }
     for (int64_t i = 0; i < nblk; ++i) {
         const int stg = static_cast<int>(i % Gm::kStages);
-        if (!mbar_wait(bars + 8u * stg, static_cast<uint32_t>((i / Gm::kStages) & 1), nullptr)) {
+        if (!mbar_wait(bars + 8u * stg, static_cast<uint32_t>((i / Gm::kStages) & 1), nullptr,
+                       i == 0 && wt.withhold ? wt.timeout_ns : kWaitTimeoutNs)) {
             // Give the copies still in flight one more bounded wait before the
             // CTA moves on (and later reuses this shared memory).
             for (int64_t j = i + 1; j < nblk && j < i + Gm::kStages; ++j)
@@ -233,7 +384,9 @@ __device__ bool warp_stream(DecState<G>& st, const uint64_t (&q2)[G][4], const b
     return true;
 }
 
-template <int D, int G>
+// Fp8: the retrieval pools hold E4M3 codes (one instantiation per format, so
+// the bf16 kernel carries no code of the other path).
+template <int D, int G, bool Fp8>
 __device__ __forceinline__ void decode_body(const DecodeParams& p) {
     using Gm = Geom<D, G>;
     constexpr int LPR = Gm::LPR;
@@ -319,16 +472,40 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
     // kernel reads or writes comes after the wait.
     if (lane == 0 && w0 < w1) {
         const int64_t pre = (w1 - w0 < kPrefetchRows<D>) ? (w1 - w0) : kPrefetchRows<D>;
-        const uint32_t bytes = static_cast<uint32_t>(pre * D * 2);
-        bulk_prefetch_l2(kbase + w0 * D, bytes);
-        bulk_prefetch_l2(vbase + w0 * D, bytes);
+        if (Fp8 && is_retr) {  // rows of one-byte codes
+            const uint32_t bytes = static_cast<uint32_t>(pre * D);
+            bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.pools.rk) + (kbase - p.pools.rk) + w0 * D, bytes);
+            bulk_prefetch_l2(reinterpret_cast<const uint8_t*>(p.pools.rv) + (vbase - p.pools.rv) + w0 * D, bytes);
+        } else {
+            const uint32_t bytes = static_cast<uint32_t>(pre * D * 2);
+            bulk_prefetch_l2(kbase + w0 * D, bytes);
+            bulk_prefetch_l2(vbase + w0 * D, bytes);
+        }
     }
     grid_dependency_wait();
     grid_launch_dependents();
 
-    // Append the new token (D1): warp 1 copies it into its slot.
+    // E4M3 retrieval cache: this head's scales; k_scale is folded into the
+    // queries, v_scale into the partial output.
+    const bool fp8 = Fp8 && is_retr;
+    const float k_scale = fp8 ? p.kv_scale[g * 4 + 0] : 1.f;
+    const float v_scale = fp8 ? p.kv_scale[g * 4 + 1] : 1.f;
+    const float k_inv = fp8 ? p.kv_scale[g * 4 + 2] : 1.f;
+    const float v_inv = fp8 ? p.kv_scale[g * 4 + 3] : 1.f;
+    // Codes of this lane's 8 elements of the new K (or V) row.
+    auto quantize8 = [&](const bf16* src, float inv) -> uint2 { return e4m3x8_from_bf16x8(ld_nc_v4(src), inv); };
+
+    // Append the new token (D1): warp 1 copies (or quantizes) it into its slot.
     if (owns_new && warp == 1) {
-        if (lane < LPR) {
+        if (fp8) {
+            uint8_t* k8 = reinterpret_cast<uint8_t*>(p.pools.rk) + (new_k_dst - p.pools.rk);
+            uint8_t* v8 = reinterpret_cast<uint8_t*>(p.pools.rv) + (new_v_dst - p.pools.rv);
+            if (lane < LPR) {
+                *reinterpret_cast<uint2*>(k8 + lane * 8) = quantize8(knew + lane * 8, k_inv);
+            } else if (lane < 2 * LPR) {
+                *reinterpret_cast<uint2*>(v8 + (lane - LPR) * 8) = quantize8(vnew + (lane - LPR) * 8, v_inv);
+            }
+        } else if (lane < LPR) {
             *reinterpret_cast<uint4*>(new_k_dst + lane * 8) = ld_nc_v4(knew + lane * 8);
         } else if (lane < 2 * LPR) {
             *reinterpret_cast<uint4*>(new_v_dst + (lane - LPR) * 8) = ld_nc_v4(vnew + (lane - LPR) * 8);
@@ -343,19 +520,34 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
         const uint32_t w[4] = {qx.x, qx.y, qx.z, qx.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            q2[h][i] = f2pack(bf16lo_to_f32(w[i]) * p.scale_log2, bf16hi_to_f32(w[i]) * p.scale_log2);
+            q2[h][i] = f2pack(bf16lo_to_f32(w[i]) * p.scale_log2 * k_scale, bf16hi_to_f32(w[i]) * p.scale_log2 * k_scale);
     }
 
     DecState<G> st;
     init_state(st);
     bool ok = true;
-    if (w0 < w1) ok = warp_stream<D, G>(st, q2, kbase, vbase, w0, w1, skip, ring, bars);
+    const WaitTest wt{p.test_withhold != 0 && blockIdx.x == 0 && warp == 0, p.test_timeout_ns};
+    if (w0 < w1) {
+        if (fp8) {
+            const uint8_t* k8 = reinterpret_cast<const uint8_t*>(p.pools.rk) + (kbase - p.pools.rk);
+            const uint8_t* v8 = reinterpret_cast<const uint8_t*>(p.pools.rv) + (vbase - p.pools.rv);
+            ok = warp_stream8<D, G>(st, q2, k8, v8, w0, w1, ring, bars, wt);
+        } else {
+            ok = warp_stream<D, G>(st, q2, kbase, vbase, w0, w1, skip, ring, bars, wt);
+        }
+    }
     if (!ok && lane == 0) atomicOr(p.err, kErrDecodeCopy);
     if (owns_new && warp == 0) {
-        uint4 kx[1] = {ld_nc_v4(knew + sub * 8)};
-        uint4 vx[1] = {ld_nc_v4(vnew + sub * 8)};
         bool valid[1] = {lane < LPR};
-        accumulate<D, G, 1>(st, q2, kx, vx, valid);
+        if (fp8) {  // the stored codes, as every later step reads them
+            uint2 kc[1] = {quantize8(knew + sub * 8, k_inv)};
+            uint2 vc[1] = {quantize8(vnew + sub * 8, v_inv)};
+            accumulate8<D, G, 1>(st, q2, kc, vc, valid);
+        } else {
+            uint4 kx[1] = {ld_nc_v4(knew + sub * 8)};
+            uint4 vx[1] = {ld_nc_v4(vnew + sub * 8)};
+            accumulate<D, G, 1>(st, q2, kx, vx, valid);
+        }
     }
 
     // Merge the row groups of the warp, then the warps.
@@ -397,9 +589,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
             O += f * sm_o[(w * G + h) * D + d];
         }
         if (final_now) {
-            p.out[(static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d] = __float2bfloat16_rn(O / Lsum);
+            p.out[(static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d] = __float2bfloat16_rn(O * v_scale / Lsum);
         } else {
-            p.part_o[(item * G + h) * D + d] = Lsum > 0.f ? O / Lsum : 0.f;
+            p.part_o[(item * G + h) * D + d] = Lsum > 0.f ? O * v_scale / Lsum : 0.f;
             if (d == 0) p.part_lse[item * G + h] = Lsum > 0.f ? M + __log2f(Lsum) : -INFINITY;
         }
     }
@@ -489,16 +681,16 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
 
 // The kernel, with the register budget its residency needs: three CTAs per SM
 // for G = 2 and 4, the compiler's own choice otherwise.
-template <int D, int G>
+template <int D, int G, bool Fp8>
 __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams p) {
-    decode_body<D, G>(p);
+    decode_body<D, G, Fp8>(p);
 }
-template <int D, int G>
+template <int D, int G, bool Fp8>
 __global__ void __launch_bounds__(kDecodeThreads, 3) decode_kernel_3(const DecodeParams p) {
-    decode_body<D, G>(p);
+    decode_body<D, G, Fp8>(p);
 }
 
-template <int D, int G>
+template <int D, int G, bool Fp8>
 cudaError_t launch_dg(const DecodeParams& p, unsigned grid, cudaStream_t s) {
     constexpr int smem = Geom<D, G>::kSmem;
     static_assert((kWarps * 2 * G + kWarps * G * D) * 4 <= Geom<D, G>::kRingBytes, "warp merge arrays fit in the ring");
@@ -507,25 +699,30 @@ cudaError_t launch_dg(const DecodeParams& p, unsigned grid, cudaStream_t s) {
     static SmemLimitOnce limit;
     static_assert(decode_ctas_per_sm(G) == 2 || decode_ctas_per_sm(G) == 3, "one of the two kernels");
     if constexpr (decode_ctas_per_sm(G) == 3) {
-        const cudaError_t e = limit.apply(reinterpret_cast<const void*>(&decode_kernel_3<D, G>), smem);
+        const cudaError_t e = limit.apply(reinterpret_cast<const void*>(&decode_kernel_3<D, G, Fp8>), smem);
         if (e != cudaSuccess) return e;
-        return launch_pdl(decode_kernel_3<D, G>, dim3(grid), dim3(kDecodeThreads), smem, s, p);
+        return launch_pdl(decode_kernel_3<D, G, Fp8>, dim3(grid), dim3(kDecodeThreads), smem, s, p);
     } else {
-        const cudaError_t e = limit.apply(reinterpret_cast<const void*>(&decode_kernel<D, G>), smem);
+        const cudaError_t e = limit.apply(reinterpret_cast<const void*>(&decode_kernel<D, G, Fp8>), smem);
         if (e != cudaSuccess) return e;
-        return launch_pdl(decode_kernel<D, G>, dim3(grid), dim3(kDecodeThreads), smem, s, p);
+        return launch_pdl(decode_kernel<D, G, Fp8>, dim3(grid), dim3(kDecodeThreads), smem, s, p);
+    }
+}
+
+template <int D, bool Fp8>
+cudaError_t launch_df(const DecodeParams& p, unsigned grid, cudaStream_t s) {
+    switch (p.G) {
+        case 1: return launch_dg<D, 1, Fp8>(p, grid, s);
+        case 2: return launch_dg<D, 2, Fp8>(p, grid, s);
+        case 4: return launch_dg<D, 4, Fp8>(p, grid, s);
+        case 8: return launch_dg<D, 8, Fp8>(p, grid, s);
+        default: return cudaErrorInvalidValue;
     }
 }
 
 template <int D>
 cudaError_t launch_d(const DecodeParams& p, unsigned grid, cudaStream_t s) {
-    switch (p.G) {
-        case 1: return launch_dg<D, 1>(p, grid, s);
-        case 2: return launch_dg<D, 2>(p, grid, s);
-        case 4: return launch_dg<D, 4>(p, grid, s);
-        case 8: return launch_dg<D, 8>(p, grid, s);
-        default: return cudaErrorInvalidValue;
-    }
+    return p.fp8 ? launch_df<D, true>(p, grid, s) : launch_df<D, false>(p, grid, s);
 }
 
 }  // namespace

@@ -116,6 +116,8 @@ extern "C" duo_status duo_decode_static_scratch(duo_cache* c, int32_t layer, con
     p.R = L.recent;
     p.W = c->W;
     p.scale_log2 = c->scale * 1.4426950408889634f;
+    p.fp8 = c->fp8 ? 1 : 0;
+    p.kv_scale = c->fp8 ? c->kv_scales + static_cast<size_t>(layer) * L.num_kv_heads * 4 : nullptr;
     std::memset(&p.heads, 0, sizeof(p.heads));
     for (int g = 0; g < L.num_kv_heads; ++g) {
         const size_t i = static_cast<size_t>(layer) * L.num_kv_heads + g;

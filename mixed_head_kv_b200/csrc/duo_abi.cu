@@ -20,7 +20,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Byte sizes of the regions of the cache buffer, in carving order.
 struct Regions {
-    size_t retr_pool, strm_pool, part_o, part_lse, counters, err, total;
+    size_t retr_pool, strm_pool, part_o, part_lse, counters, err, scales, total;
 };
 
 // Split-KV partials are written by retrieval (b, KV head, split) items only, indexed
@@ -31,14 +31,20 @@ Regions regions_for(const duo_layout& L, int64_t n_retr_all, int64_t n_strm_all,
     const size_t D = static_cast<size_t>(L.head_dim);
     const size_t W = static_cast<size_t>(L.sink) + static_cast<size_t>(L.recent);
     const size_t G = static_cast<size_t>(L.num_q_heads / L.num_kv_heads);
-    r.retr_pool = align_up(static_cast<size_t>(n_retr_all) * L.batch * static_cast<size_t>(L.max_len) * D * 2);
+    const size_t retr_elem = L.kv_format == DUO_KV_E4M3 ? 1 : 2;  // E4M3 codes or bf16
+    r.retr_pool =
+        align_up(static_cast<size_t>(n_retr_all) * L.batch * static_cast<size_t>(L.max_len) * D * retr_elem);
     r.strm_pool = align_up(static_cast<size_t>(n_strm_all) * L.batch * W * D * 2);
     const size_t items = static_cast<size_t>(L.batch) * static_cast<size_t>(max_retr_layer) * kDecodeMaxSplits;
     r.part_o = align_up(items * G * D * sizeof(float));
     r.part_lse = align_up(items * G * sizeof(float));
     r.counters = align_up(static_cast<size_t>(L.batch) * L.num_kv_heads * sizeof(uint32_t));
     r.err = align_up(sizeof(uint32_t));
-    r.total = 2 * r.retr_pool + 2 * r.strm_pool + r.part_o + r.part_lse + r.counters + r.err;
+    // E4M3 caches: k_scale, v_scale and their reciprocals per (layer, KV head)
+    r.scales = L.kv_format == DUO_KV_E4M3
+                   ? align_up(static_cast<size_t>(L.num_layers) * L.num_kv_heads * 4 * sizeof(float))
+                   : 0;
+    r.total = 2 * r.retr_pool + 2 * r.strm_pool + r.part_o + r.part_lse + r.counters + r.err + r.scales;
     return r;
 }
 
@@ -55,6 +61,7 @@ duo_status check_layout(const duo_layout* L, const uint8_t* mask) {
     if (static_cast<int64_t>(L->sink) + L->recent > (1 << 30)) return DUO_ERR_INVALID_ARG;
     if (L->max_len < 1 || L->max_len > (int64_t{1} << 31) - 1) return DUO_ERR_INVALID_ARG;
     if (!(L->softmax_scale >= 0.f) || !std::isfinite(L->softmax_scale)) return DUO_ERR_INVALID_ARG;
+    if (L->kv_format != DUO_KV_BF16 && L->kv_format != DUO_KV_E4M3) return DUO_ERR_INVALID_ARG;
     const int64_t n = static_cast<int64_t>(L->num_layers) * L->num_kv_heads;
     for (int64_t i = 0; i < n; ++i)
         if (mask[i] > 1) return DUO_ERR_INVALID_ARG;
@@ -199,26 +206,42 @@ duo_status duo_cache_alloc(const duo_layout* layout, const uint8_t* is_retrieval
     c->part_o = reinterpret_cast<float*>(p); p += reg.part_o;
     c->part_lse = reinterpret_cast<float*>(p); p += reg.part_lse;
     c->counters = reinterpret_cast<uint32_t*>(p); p += reg.counters;
-    c->err = reinterpret_cast<uint32_t*>(p);
+    c->err = reinterpret_cast<uint32_t*>(p); p += reg.err;
+    c->fp8 = L.kv_format == DUO_KV_E4M3;
+    c->kv_scales = c->fp8 ? reinterpret_cast<float*>(p) : nullptr;
 
-    // Pool tensor maps; an empty pool gets a map over the other pool (never read).
+    // Pool tensor maps (bf16 tiles for the prefill kernel). An empty pool gets a
+    // map over the other pool, never read; so does an E4M3 retrieval pool, whose
+    // cache tiles prefill never reads (it refuses such chunks). A cache with no
+    // bf16 pool at all (every head an E4M3 retrieval head) needs no map.
     const int64_t D = L.head_dim;
-    const void* rk = nr ? static_cast<const void*>(c->pools.rk) : c->pools.sk;
-    const void* rv = nr ? static_cast<const void*>(c->pools.rv) : c->pools.sv;
+    const bool bf16_retr = nr > 0 && !c->fp8;
+    const bool any_bf16 = bf16_retr || ns > 0;
+    const void* rk = bf16_retr ? static_cast<const void*>(c->pools.rk) : c->pools.sk;
+    const void* rv = bf16_retr ? static_cast<const void*>(c->pools.rv) : c->pools.sv;
     const void* sk = ns ? static_cast<const void*>(c->pools.sk) : c->pools.rk;
     const void* sv = ns ? static_cast<const void*>(c->pools.sv) : c->pools.rv;
-    const int64_t rslots = nr ? L.max_len : c->W;
+    const int64_t rslots = bf16_retr ? L.max_len : c->W;
     const int64_t sslots = ns ? c->W : L.max_len;
-    const int64_t rz = static_cast<int64_t>(nr ? nr : ns) * L.batch;
+    const int64_t rz = static_cast<int64_t>(bf16_retr ? nr : ns) * L.batch;
     const int64_t sz = static_cast<int64_t>(ns ? ns : nr) * L.batch;
-    if (!make_pool_map(&c->map_rk, rk, D, rslots, rz) || !make_pool_map(&c->map_rv, rv, D, rslots, rz) ||
-        !make_pool_map(&c->map_sk, sk, D, sslots, sz) || !make_pool_map(&c->map_sv, sv, D, sslots, sz)) {
+    if (any_bf16 &&
+        (!make_pool_map(&c->map_rk, rk, D, rslots, rz) || !make_pool_map(&c->map_rv, rv, D, rslots, rz) ||
+         !make_pool_map(&c->map_sk, sk, D, sslots, sz) || !make_pool_map(&c->map_sv, sv, D, sslots, sz))) {
         delete c;
         return DUO_ERR_CUDA;
     }
     if (cudaMemsetAsync(dev_buf, 0, reg.total, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
         delete c;
         return DUO_ERR_CUDA;
+    }
+    if (c->fp8) {  // scale 1 for every head until duo_cache_set_kv_scales
+        c->kv_scales_host.assign(static_cast<size_t>(L.num_layers) * L.num_kv_heads * 4, 1.0f);
+        if (cudaMemcpyAsync(c->kv_scales, c->kv_scales_host.data(), c->kv_scales_host.size() * sizeof(float),
+                            cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+            delete c;
+            return DUO_ERR_CUDA;
+        }
     }
     // Decode parameters that do not change between steps, per layer.
     c->decode_tmpl.assign(L.num_layers, DecodeParams{});
@@ -239,6 +262,8 @@ duo_status duo_cache_alloc(const duo_layout* layout, const uint8_t* is_retrieval
         t.R = L.recent;
         t.W = c->W;
         t.scale_log2 = c->scale * 1.4426950408889634f;
+        t.fp8 = c->fp8 ? 1 : 0;
+        t.kv_scale = c->fp8 ? c->kv_scales + static_cast<size_t>(layer) * L.num_kv_heads * 4 : nullptr;
         fill_heads(c, layer, &t.heads);
         for (int g = 0; g < L.num_kv_heads; ++g) {
             if (t.heads.is_retr[g]) t.retr_list[t.n_retr++] = static_cast<int16_t>(g);
@@ -273,6 +298,35 @@ duo_status duo_cache_set_len(duo_cache* c, int32_t layer, int64_t len) {
     return DUO_OK;
 }
 
+duo_status duo_cache_set_kv_scales(duo_cache* c, int32_t layer, const float* k_scale, const float* v_scale,
+                                   void* stream) {
+    if (!c || !k_scale || !v_scale || layer < 0 || layer >= c->lay.num_layers) return DUO_ERR_INVALID_ARG;
+    if (!c->fp8) return DUO_ERR_STATE;
+    const int32_t H = c->lay.num_kv_heads;
+    for (int32_t g = 0; g < H; ++g)
+        if (!(k_scale[g] > 0.f) || !(v_scale[g] > 0.f) || !std::isfinite(k_scale[g]) || !std::isfinite(v_scale[g]))
+            return DUO_ERR_INVALID_ARG;
+    float* h = c->kv_scales_host.data() + static_cast<size_t>(layer) * H * 4;
+    for (int32_t g = 0; g < H; ++g) {
+        h[g * 4 + 0] = k_scale[g];
+        h[g * 4 + 1] = v_scale[g];
+        h[g * 4 + 2] = 1.0f / k_scale[g];  // fp32 reciprocals: the quantizer multiplies by them
+        h[g * 4 + 3] = 1.0f / v_scale[g];
+    }
+    if (cudaMemcpyAsync(c->kv_scales + static_cast<size_t>(layer) * H * 4, h, static_cast<size_t>(H) * 4 * sizeof(float),
+                        cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return DUO_ERR_CUDA;
+    return DUO_OK;
+}
+
+duo_status duo_cache_test_wait_timeout(duo_cache* c, int32_t launches, uint64_t timeout_ns) {
+    if (!c || (launches & ~(DUO_TEST_WAIT_DECODE | DUO_TEST_WAIT_PREFILL)) != 0) return DUO_ERR_INVALID_ARG;
+    if (timeout_ns < 1000 || timeout_ns > 1000000000ull) return DUO_ERR_INVALID_ARG;
+    c->test_wait = launches;
+    c->test_wait_ns = timeout_ns;
+    return DUO_OK;
+}
+
 duo_status duo_cache_seq_lens(const duo_cache* c, int32_t layer, int64_t* lens) {
     if (!c || !lens || layer < 0 || layer >= c->lay.num_layers) return DUO_ERR_INVALID_ARG;
     const int64_t* L = seq_lens(c, layer);
@@ -297,9 +351,14 @@ duo_status duo_cache_views(const duo_cache* c, int32_t layer, int32_t kv_head, v
     const int64_t D = c->lay.head_dim;
     const bool r = c->is_retr[i] != 0;
     const int64_t nslots = r ? c->lay.max_len : c->W;
-    const int64_t off = static_cast<int64_t>(c->pool_idx[i]) * c->lay.batch * nslots * D;
-    if (k) *k = (r ? c->pools.rk : c->pools.sk) + off;
-    if (v) *v = (r ? c->pools.rv : c->pools.sv) + off;
+    const int64_t off = static_cast<int64_t>(c->pool_idx[i]) * c->lay.batch * nslots * D;  // elements
+    if (r && c->fp8) {  // one byte per element
+        if (k) *k = reinterpret_cast<uint8_t*>(c->pools.rk) + off;
+        if (v) *v = reinterpret_cast<uint8_t*>(c->pools.rv) + off;
+    } else {
+        if (k) *k = (r ? c->pools.rk : c->pools.sk) + off;
+        if (v) *v = (r ? c->pools.rv : c->pools.sv) + off;
+    }
     if (slots) *slots = nslots;
     if (is_retrieval) *is_retrieval = r ? 1 : 0;
     return DUO_OK;
@@ -351,6 +410,8 @@ duo_status append_impl(duo_cache* c, int32_t layer, const void* k, const void* v
     p.S = c->lay.sink;
     p.R = c->lay.recent;
     p.W = c->W;
+    p.fp8 = c->fp8 ? 1 : 0;
+    p.kv_scale = c->fp8 ? c->kv_scales + static_cast<size_t>(layer) * c->lay.num_kv_heads * 4 : nullptr;
     p.ragged = uniform ? 0 : 1;
     if (!uniform) {
         for (int32_t b = 0; b < B; ++b) {
@@ -407,6 +468,13 @@ duo_status prefill_impl(duo_cache* c, int32_t layer, const void* q, const void* 
     if (!q || !k || !v || !out) return DUO_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DUO_ERR_ALIGNMENT;
     if (!uniform && B > kMaxRaggedBatch) return DUO_ERR_STATE;
+    if (c->fp8) {  // the tensor-core prefill reads bf16 cache tiles only
+        bool has_retr = false;
+        for (int32_t g = 0; g < c->lay.num_kv_heads; ++g)
+            has_retr = has_retr || c->is_retr[static_cast<size_t>(layer) * c->lay.num_kv_heads + g];
+        for (int32_t b = 0; b < B && has_retr; ++b)
+            if (lens[b] > 0) return DUO_ERR_STATE;
+    }
     const int64_t n_rows = max_tok;  // rows per sequence of the padded tensors
     const int64_t len0 = lens[0];
     const duo_layout& L = c->lay;
@@ -451,7 +519,12 @@ duo_status prefill_impl(duo_cache* c, int32_t layer, const void* q, const void* 
         !make_chunk_map(&maps.k, k, L.head_dim, L.num_kv_heads, n_rows, L.batch) ||
         !make_chunk_map(&maps.v, v, L.head_dim, L.num_kv_heads, n_rows, L.batch))
         return DUO_ERR_CUDA;
-    if (launch_prefill(p, maps, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUO_ERR_CUDA;
+    if (c->test_wait & DUO_TEST_WAIT_PREFILL) {  // one launch only
+        p.test_withhold = 1;
+        p.test_timeout_ns = c->test_wait_ns;
+        c->test_wait &= ~DUO_TEST_WAIT_PREFILL;
+    }
+    if (launch_prefill(p, maps, c->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUO_ERR_CUDA;
     return DUO_OK;
 }
 
@@ -485,6 +558,11 @@ duo_status duo_decode(duo_cache* c, int32_t layer, const void* q, const void* k_
     p.k_new = static_cast<const bf16*>(k_new);
     p.v_new = static_cast<const bf16*>(v_new);
     p.out = static_cast<bf16*>(out);
+    if (c->test_wait & DUO_TEST_WAIT_DECODE) {  // one launch only
+        p.test_withhold = 1;
+        p.test_timeout_ns = c->test_wait_ns;
+        c->test_wait &= ~DUO_TEST_WAIT_DECODE;
+    }
     const int64_t rows = p.len + 1;
     const int64_t nsplit = decode_plan(c, layer, rows);
     p.split_rows = (rows + nsplit - 1) / nsplit;

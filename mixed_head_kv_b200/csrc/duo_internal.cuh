@@ -78,6 +78,8 @@ struct AppendParams {
     int32_t B, Hkv, D, S, R, W;
     int32_t ragged;   // 1: per-sequence seq_len / seq_n below
     int32_t n_retr;   // retrieval KV heads of the layer, listed first in order[]
+    int32_t fp8;            // retrieval pools hold E4M3 codes
+    const float* kv_scale;  // fp8: [Hkv][k_scale, v_scale, 1/k_scale, 1/v_scale] of this layer
     HeadMap heads;
     int16_t order[DUO_MAX_KV_HEADS];   // KV heads, retrieval heads first
     int64_t seq_len[kMaxRaggedBatch];  // tokens cached before this call, per sequence
@@ -146,6 +148,10 @@ struct DecodeParams {
     int16_t strm_list[DUO_MAX_KV_HEADS];
     HeadMap heads;
     int32_t ragged;                     // 1: per-sequence lengths in seq_len
+    int32_t fp8;                        // retrieval pools hold E4M3 codes
+    const float* kv_scale;              // fp8: [Hkv][k_scale, v_scale, 1/k_scale, 1/v_scale] of this layer
+    int32_t test_withhold;              // 1: a test of the bounded waits (duo_cache_test_wait_timeout)
+    uint64_t test_timeout_ns;           // the withheld copy's wait limit
     int64_t seq_len[kMaxRaggedBatch];   // tokens cached before this step, per sequence
 };
 cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
@@ -166,6 +172,8 @@ struct PrefillParams {
     int16_t qhead[DUO_MAX_Q_HEADS];
     HeadMap heads;
     int32_t ragged;                    // 1: per-sequence seq_len / seq_c below
+    int32_t test_withhold;             // 1: a test of the bounded waits (duo_cache_test_wait_timeout)
+    uint64_t test_timeout_ns;          // the withheld copy's wait limit
     int64_t seq_len[kMaxRaggedBatch];  // tokens cached before the chunk, per sequence
     int32_t seq_c[kMaxRaggedBatch];    // chunk rows that are tokens, per sequence (<= C)
 };
@@ -179,7 +187,7 @@ struct PrefillMaps {
     CUtensorMap sk;  // streaming pool (D, W, n_strm_all*B), box (64, 128, 1)
     CUtensorMap sv;
 };
-cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t s);
+cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, int num_sms, cudaStream_t s);
 
 }  // namespace duo
 
@@ -201,6 +209,11 @@ struct duo_cache {
     uint32_t* counters = nullptr;
     uint32_t* err = nullptr;
     CUtensorMap map_rk{}, map_rv{}, map_sk{}, map_sv{};
+    int32_t test_wait = 0;              // duo_cache_test_wait_timeout: launch kinds still to withhold a copy
+    uint64_t test_wait_ns = 0;
+    bool fp8 = false;                   // retrieval pools hold E4M3 codes
+    float* kv_scales = nullptr;         // device [layers][Hkv][k_scale, v_scale, 1/k_scale, 1/v_scale]
+    std::vector<float> kv_scales_host;  // host copy of kv_scales
     std::vector<duo::DecodeParams> decode_tmpl;  // [layers] decode parameters fixed at alloc
     std::vector<int64_t> plan_key;               // [layers] rows / 256 of the cached split plan
     std::vector<int64_t> plan_nsplit;            // [layers] the plan's split count

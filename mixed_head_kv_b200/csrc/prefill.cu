@@ -192,6 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ring = is_k ? sK : sV;
             const int full = is_k ? kKFull : kVFull;
             const int empty = is_k ? kKEmpty : kVEmpty;
+            // Test of the bounded waits: CTA 0 never issues its first K tile.
+            const bool withhold = is_k && p.test_withhold != 0 && blockIdx.x == 0;
             int issued = 0;  // tiles whose load was issued
             for (int j = 0; j < n; ++j) {
                 const int st = j & 1;
@@ -205,17 +207,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     record_abort(p.err, abort_flag);
                     break;
                 }
+                issued = j + 1;
+                if (withhold && j == 0) continue;
                 mbar_arrive_expect_tx(bar(full + st), Lay::kTile);
                 for (int kb = 0; kb < Lay::kColBlocks; ++kb) {
                     const uint32_t dst = ring + st * Lay::kTile + kb * kTileBytesPerColBlock;
                     if (src == 2) tma_load_4d(dst, m, bar(full + st), kb * 64, it.g, row0, it.b);
                     else tma_load_3d(dst, m, bar(full + st), kb * 64, row0, zpool);
                 }
-                issued = j + 1;
             }
             // Let every load this thread issued land before the CTA can exit.
             for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-                mbar_wait(bar(full + (j & 1)), (j >> 1) & 1, nullptr);
+                if (!(withhold && j == 0)) mbar_wait(bar(full + (j & 1)), (j >> 1) & 1, nullptr);
         }
     } else if (warp == 9) {
         // ------------------------------------------------------------ MMA issuer
@@ -225,7 +228,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // S(j) = Q K(j)^T into S buffer j&1.
             auto qk = [&](int j) -> bool {
                 const int st = j & 1;
-                if (!mbar_wait(bar(kKFull + st), (j >> 1) & 1, abort_flag)) return false;
+                const bool withheld = j == 0 && p.test_withhold != 0 && blockIdx.x == 0;
+                if (!mbar_wait(bar(kKFull + st), (j >> 1) & 1, abort_flag,
+                               withheld ? p.test_timeout_ns : kWaitTimeoutNs))
+                    return false;
                 tc_fence_after();
                 const uint32_t kt = sK + st * Lay::kTile;
 #pragma unroll
@@ -446,7 +452,7 @@ cudaError_t launch_d(const PrefillParams& p, const PrefillMaps& maps, cudaStream
 
 }  // namespace
 
-cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t s) {
+cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, int /*num_sms*/, cudaStream_t s) {
     if (p.B * p.Hq * p.n_qt == 0) return cudaSuccess;
     if (p.D == 128) return launch_d<128>(p, maps, s);
     if (p.D == 64) return launch_d<64>(p, maps, s);

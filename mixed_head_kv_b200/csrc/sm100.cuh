@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace duo {
 
@@ -14,7 +15,7 @@ namespace duo {
 // an error in the cache's error word and unwinds instead of hanging the GPU.
 constexpr uint64_t kWaitTimeoutNs = 1000000000ull;  // 1 s
 
-// Error-word bits written by kernels.
+// Error-word bits written by kernels (DUO_ERR_BIT_* in duo.h).
 constexpr uint32_t kErrPrefillWait = 1u << 0;
 constexpr uint32_t kErrDecodeCopy = 1u << 1;
 
@@ -62,14 +63,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed. Returns false if
-// `abort_flag` (may be null) becomes non-zero or kWaitTimeoutNs elapses first.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag) {
+// `abort_flag` (may be null) becomes non-zero or `timeout_ns` elapses first.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag,
+                                          uint64_t timeout_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (abort_flag != nullptr && *abort_flag) return false;
-        if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+        if (global_timer_ns() - t0 > timeout_ns) return false;
     }
 }
 
@@ -113,6 +115,12 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 r;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+    return r;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 r;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
     return r;
 }
 
@@ -237,6 +245,33 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ---------------------------------------------------------------- FP8 E4M3
+// E4M3 codes of (lo, hi) in one 16-bit word, lo in the low byte: the hardware
+// conversion, round to nearest even, saturating to +-448.
+__device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Values of the two E4M3 codes of a 16-bit word (low byte -> lo); exact in f16.
+__device__ __forceinline__ void e4m3x2_to_f32(uint16_t c, float& lo, float& hi) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+    lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+    hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+}
+
+// Codes of eight bf16 values (16 bytes) times `inv` (the product in fp32), as 8 bytes.
+__device__ __forceinline__ uint2 e4m3x8_from_bf16x8(const uint4& x, float inv) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t c[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        c[j] = e4m3x2_from_f32(__uint_as_float(w[j] << 16) * inv, __uint_as_float(w[j] & 0xFFFF0000u) * inv);
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
 
 // ---------------------------------------------------------------- packed fp32 pairs
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {

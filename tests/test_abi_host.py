@@ -127,3 +127,14 @@ def test_status_strings():
     for s in range(8):
         assert duo.duo_status_str(s) and duo.duo_status_str(s) != "unknown status"
     assert duo.duo_status_str(99) == "unknown status"
+
+
+def test_e4m3_cache_sizes():
+    """E4M3 retrieval pools take one byte per element instead of two; the cache
+    gains a region of 4 fp32 scales per (layer, KV head)."""
+    mask = [1, 0, 1, 0, 1, 1, 0, 0]
+    _, b16, _ = duo.duo_cache_alloc(duo.make_layout(2, 1, 8, 4, 128, 64, 256, 4096), mask)
+    _, b8, _ = duo.duo_cache_alloc(duo.make_layout(2, 1, 8, 4, 128, 64, 256, 4096, kv_format=duo.DUO_KV_E4M3), mask)
+    assert b16 - b8 == 2 * 4 * 4096 * 128 - 256
+    st, _, _ = duo.duo_cache_alloc(duo.make_layout(2, 1, 8, 4, 128, 64, 256, 4096, kv_format=2), mask)
+    assert st == duo.DUO_ERR_INVALID_ARG
