@@ -742,9 +742,15 @@ def secondary_cases():
     return cases
 
 
-def run_secondary(duo, peaks, emit=None):
+def case_name(kind, w):
+    return w.name + ("_e4m3" if kind == "decode_e4m3" else "")
+
+
+def run_secondary(duo, peaks, emit=None, only=None):
     out = []
     for kind, w, layers, steps in secondary_cases():
+        if only is not None and case_name(kind, w) not in only:
+            continue
         if kind == "prefill":
             case = PrefillCase(duo, w)
         else:
@@ -767,7 +773,7 @@ def run_sweep(args):
     import __graft_entry__
     __graft_entry__.build()
     import mixed_head_kv_b200 as duo
-    return run_secondary(duo, load_peaks(), emit=lambda d: print(json.dumps(d), flush=True))
+    return run_secondary(duo, load_peaks(), emit=lambda d: print(json.dumps(d), flush=True), only=args.case)
 
 
 # ----------------------------------------------------------------------------- memory footprint
@@ -815,6 +821,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--sweep", action="store_true",
                     help="time only the other workloads (GQA decode at 128K and 1M, MHA ratio sweep), a line each")
+    ap.add_argument("--case", action="append", default=None,
+                    help="with --sweep: only this workload (repeatable), e.g. llama3_8b_gqa_128k_decode_b4_e4m3")
     ap.add_argument("--no-secondary", action="store_true",
                     help="leave the other workloads out of the main line (they run by default at N=1)")
     ap.add_argument("--memory", action="store_true",

@@ -322,23 +322,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             tile_of(it, j, src, row0);
             const bool full =
                 it.retr && ((src == 0 && row0 + kTileK <= it.L) || (src == 2 && row0 + kTileK <= it.q0));
+            // Each 32-key word of this half: masked element-wise only when some lane
+            // of the warp sees part of it; skipped altogether (no max, no exp2, P = 0)
+            // when no lane of the warp sees any of its keys. Both tests are
+            // warp-uniform, so the branches do not diverge.
+            bool live[2] = {true, true};
             if (!full) {
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
                     const uint32_t bits = visible_bits(p, it, src, row0, 2 * h + w, qrow, ring);
+                    live[w] = __any_sync(0xffffffffu, bits != 0u);
+                    if (live[w] && !__all_sync(0xffffffffu, bits == 0xFFFFFFFFu)) {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        if (!((bits >> k) & 1u)) s[w * 32 + k] = -INFINITY;
+                        for (int k = 0; k < 32; ++k)
+                            if (!((bits >> k) & 1u)) s[w * 32 + k] = -INFINITY;
+                    }
                 }
             }
             float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-            static_assert(kHalf % 8 == 0, "the max loop covers exactly [0, kHalf)");
+            static_assert(kHalf == 64, "two 32-key words per softmax thread and tile");
 #pragma unroll
-            for (int i = 0; i < kHalf; i += 8) {
-                m0 = fmax3(m0, s[i], s[i + 1]);
-                m1 = fmax3(m1, s[i + 2], s[i + 3]);
-                m2 = fmax3(m2, s[i + 4], s[i + 5]);
-                m3 = fmax3(m3, s[i + 6], s[i + 7]);
+            for (int w = 0; w < 2; ++w) {
+                if (!live[w]) continue;
+#pragma unroll
+                for (int i = 32 * w; i < 32 * w + 32; i += 8) {
+                    m0 = fmax3(m0, s[i], s[i + 1]);
+                    m1 = fmax3(m1, s[i + 2], s[i + 3]);
+                    m2 = fmax3(m2, s[i + 4], s[i + 5]);
+                    m3 = fmax3(m3, s[i + 6], s[i + 7]);
+                }
             }
             const float mt = fmax3(fmaxf(m0, m1), m2, m3) * p.scale_log2;
             float factor = 1.f;
@@ -351,13 +363,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint64_t acc2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
             uint32_t pk[kHalf / 2];
 #pragma unroll
-            for (int i = 0; i < kHalf; i += 2) {
-                float e0, e1;
-                f2unpack(ffma2(f2pack(s[i], s[i + 1]), scale2, negm), e0, e1);
-                const float p0 = fast_exp2(e0);
-                const float p1 = fast_exp2(e1);
-                acc2[(i / 2) & 1] = fadd2(acc2[(i / 2) & 1], f2pack(p0, p1));
-                pk[i / 2] = pack_bf16x2(p0, p1);
+            for (int w = 0; w < 2; ++w) {
+                if (!live[w]) {
+#pragma unroll
+                    for (int i = 16 * w; i < 16 * w + 16; ++i) pk[i] = 0u;
+                    continue;
+                }
+#pragma unroll
+                for (int i = 32 * w; i < 32 * w + 32; i += 2) {
+                    float e0, e1;
+                    f2unpack(ffma2(f2pack(s[i], s[i + 1]), scale2, negm), e0, e1);
+                    const float p0 = fast_exp2(e0);
+                    const float p1 = fast_exp2(e1);
+                    acc2[(i / 2) & 1] = fadd2(acc2[(i / 2) & 1], f2pack(p0, p1));
+                    pk[i / 2] = pack_bf16x2(p0, p1);
+                }
             }
             float a0, a1;
             f2unpack(fadd2(acc2[0], acc2[1]), a0, a1);
