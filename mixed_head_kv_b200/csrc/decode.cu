@@ -727,9 +727,10 @@ cudaError_t launch_d(const DecodeParams& p, unsigned grid, cudaStream_t s) {
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeParams& p, const DecodeMaps& maps, cudaStream_t s) {
     const unsigned grid = static_cast<unsigned>(p.B * p.n_retr * p.nsplit + p.B * p.n_strm);
     if (grid == 0) return cudaSuccess;
+    if (decode_on_tensor_cores(p.G, p.D, p.fp8 != 0) && p.test_withhold == 0) return launch_decode_tc(p, maps, s);
     if (p.D == 128) return launch_d<128>(p, grid, s);
     if (p.D == 64) return launch_d<64>(p, grid, s);
     return cudaErrorInvalidValue;

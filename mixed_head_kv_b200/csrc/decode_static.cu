@@ -130,7 +130,8 @@ extern "C" duo_status duo_decode_static_scratch(duo_cache* c, int32_t layer, con
     // Same split plan as duo_decode, then limited to what the array holds.
     const int64_t rows = p.len + 1;
     int64_t nsplit =
-        plan_decode_splits(L.batch, p.n_retr, p.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms, c->G);
+        plan_decode_splits(L.batch, p.n_retr, p.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms, c->G, p.D,
+                           p.fp8 != 0);
     const size_t counters_bytes = round256(static_cast<size_t>(L.batch) * L.num_kv_heads * sizeof(uint32_t));
     if (p.n_retr > 0) {
         const int64_t pairs = static_cast<int64_t>(L.batch) * p.n_retr;
@@ -156,7 +157,7 @@ extern "C" duo_status duo_decode_static_scratch(duo_cache* c, int32_t layer, con
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(p.counters, 0, counters_bytes, s) != cudaSuccess) return DUO_ERR_CUDA;
-    if (launch_decode(p, s) != cudaSuccess) return DUO_ERR_CUDA;
+    if (launch_decode(p, decode_maps(c), s) != cudaSuccess) return DUO_ERR_CUDA;
     int64_t* lens = seq_lens(c, layer);
     for (int32_t b = 0; b < L.batch; ++b) lens[b] += 1;
     return DUO_OK;

@@ -1,0 +1,533 @@
+// decode_tc.cu — one DuoAttention decoding step on the tensor cores, for query
+// groups of G = 4 and 8 heads with head_dim 128 and bf16 caches (the group's
+// queries share every K/V row, so the per-row dot products and the P·V update
+// form small matrix products).
+//
+// Work items, one CTA each (one CTA per SM, 192 threads), the same items as the
+// CUDA-core kernel (decode.cu):
+//   retrieval (b, KV head, split): keys [s*split_rows, min((s+1)*split_rows, len+1))
+//     of the full cache; partial (o, log2-sum-exp2) to scratch, merged by the
+//     last CTA of the (b, KV head);
+//   streaming (b, KV head): the min(len+1, sink+recent) valid slots of the sink
+//     + ring cache, written straight to `out`.
+// The CTA that owns position len first writes the new token into its cache
+// slot (for a streaming head, the ring slot that held position len - recent,
+// outside the new query's window) and then reads it back with the other rows.
+//
+// Roles:
+//   warps 0-3  softmax: thread t owns key t of every 128-key tile (TMEM lane t);
+//   warp 4     TMA producer of the K and V tiles (3-stage rings, 128-B swizzle);
+//   warp 5     TMEM allocator and MMA issuer (one thread).
+// Per key tile j (keys r0 + 128j ..):
+//   S^T(j) = K(j) Q^T    M = 128 keys, N = 16 (the G query heads, zero-padded),
+//                        K = head_dim; A = the K tile (K-major), B = the queries
+//                        (K-major, built once in shared memory);
+//   P^T(j)               thread t writes the G probabilities of key t as bf16 into
+//                        a 16 x 128 K-major buffer (double-buffered);
+//   O^T += V(j)^T P^T(j) M = 128 output columns, N = 16, K = 128 keys; A = the V
+//                        tile read MN-major, B = P^T; O^T lives in TMEM (lane = column).
+// S^T is double-buffered in TMEM: QK(j+2) is issued after PV(j) (tcgen05 MMAs of
+// one thread run in issue order). The running max of each head is shared by the
+// CTA and raised only when a score exceeds it by more than 2^8 (one barrier
+// reduction per tile decides). Every mbarrier wait is time-bounded; on timeout
+// the CTA records kErrDecodeCopy, drains what it issued and unwinds.
+#include <cfloat>
+
+#include "duo_internal.cuh"
+#include "sm100.cuh"
+
+namespace duo {
+
+namespace {
+
+constexpr int kTcThreads = 192;
+constexpr int kTcD = 128;
+constexpr int kTcKeys = 128;                    // keys per tile
+constexpr int kTcN = 16;                        // query heads padded to the MMA's N
+constexpr int kTcStages = 3;
+constexpr int kTcTile = kTcKeys * kTcD * 2;     // one K or V tile: 32 KB
+constexpr int kTcColBlock = kTcKeys * 128;      // 128 rows x 128 B (64 bf16)
+constexpr int kTcQBytes = kTcN * kTcD * 2;      // 4 KB: 2 column blocks of 16 rows x 128 B
+constexpr int kTcPBytes = kTcN * kTcKeys * 2;   // 4 KB: 2 key blocks of 16 rows x 128 B
+constexpr float kTcRescale = 8.0f;
+
+// Shared-memory map (offsets from a 1024-byte-aligned base).
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kTcStages * kTcTile;
+constexpr int kOffQ = kOffV + kTcStages * kTcTile;
+constexpr int kOffP = kOffQ + kTcQBytes;                 // 2 buffers
+constexpr int kOffBar = kOffP + 2 * kTcPBytes;
+constexpr int kOffRed = kOffBar + 32 * 8;                // [2][4 warps][16 heads] floats
+constexpr int kOffMisc = kOffRed + 2 * 4 * kTcN * 4;
+constexpr int kTcSmem = kOffMisc + 64 + 1024;            // + slack for 1024-byte alignment
+static_assert(kTcSmem <= 227 * 1024, "shared memory of one CTA");
+
+// mbarriers
+constexpr int bKFull = 0;    // + stage
+constexpr int bVFull = 3;    // + stage
+constexpr int bKEmpty = 6;   // + stage
+constexpr int bVEmpty = 9;   // + stage
+constexpr int bSFull = 12;   // + S buffer
+constexpr int bPFull = 14;   // + P buffer (4 arrivals)
+constexpr int bPEmpty = 16;  // + P buffer
+constexpr int bODone = 18;   // one phase per tile
+constexpr int bOFinal = 19;
+constexpr int bDrain = 20;
+
+// TMEM columns: S^T buffers [0,16) [16,32), O^T [32,48)
+constexpr uint32_t kTcTmemCols = 64;
+constexpr uint32_t kTcTmemO = 32;
+
+// OR of a predicate over the 128 softmax threads (named barrier 1; every
+// softmax thread executes it once per tile, whatever its state).
+__device__ __forceinline__ bool softmax_any(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Byte offset of element (row, col) of a 16-row, K-major, 128-byte-swizzled
+// operand whose K extent is split into 64-element blocks of 2 KB (8-row swizzle
+// atoms of 1 KB; the 16-byte chunk index is XORed with the row within the atom).
+__device__ __forceinline__ uint32_t sw128_off16(int row, int col) {
+    const int blk = col >> 6;
+    const int chunk = (col & 63) >> 3;
+    return static_cast<uint32_t>(blk * 2048 + (row >> 3) * 1024 + (row & 7) * 128 + ((chunk ^ (row & 7)) << 4) +
+                                 (col & 7) * 2);
+}
+
+__device__ __forceinline__ void tc_abort(uint32_t* err, volatile int* abort_flag) {
+    *abort_flag = 1;
+    atomicOr(err, kErrDecodeCopy);
+}
+
+template <int G>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    decode_tc_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ DecodeMaps maps) {
+    static_assert(G <= kTcN, "query group larger than the MMA's N");
+    constexpr int D = kTcD;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* const sb = smem_raw + (base - raw);
+    auto bar = [&](int i) { return base + kOffBar + 8u * i; };
+    volatile float* red = reinterpret_cast<volatile float*>(sb + kOffRed);
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sb + kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sb + kOffMisc + 4);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(sb + kOffMisc + 8);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+
+    // Work item.
+    const int n_retr_items = p.B * p.n_retr * p.nsplit;
+    const bool is_retr = static_cast<int>(blockIdx.x) < n_retr_items;
+    int b, g, ri = 0, split = 0;
+    if (is_retr) {
+        split = blockIdx.x % p.nsplit;
+        const int t_ = blockIdx.x / p.nsplit;
+        ri = t_ % p.n_retr;
+        b = t_ / p.n_retr;
+        g = p.retr_list[ri];
+    } else {
+        const int si = blockIdx.x - n_retr_items;
+        b = si / p.n_strm;
+        g = p.strm_list[si % p.n_strm];
+    }
+    const int pool = p.heads.pool_idx[g];
+    const int64_t L = p.ragged ? p.seq_len[b] : p.len;  // this sequence's new token position
+    int64_t r0, r_end, new_slot;
+    bool owns_new;
+    if (is_retr) {
+        r0 = static_cast<int64_t>(split) * p.split_rows;
+        const int64_t s1 = r0 + p.split_rows;
+        // Splits are cut for the longest sequence: in a ragged batch a shorter
+        // sequence's last splits hold no rows (they still report to the merge).
+        owns_new = r0 <= L && s1 >= L + 1;
+        r_end = owns_new ? L + 1 : (s1 < L ? s1 : (L > r0 ? L : r0));
+        new_slot = L;
+    } else {
+        r0 = 0;
+        r_end = (L + 1 < p.W) ? (L + 1) : p.W;
+        owns_new = true;
+        new_slot = (L < p.S) ? L : p.S + (L - p.S) % p.R;
+    }
+    const int n_tiles = static_cast<int>((r_end - r0 + kTcKeys - 1) / kTcKeys);
+    const int zrow = pool * p.B + b;  // the pool map's third coordinate
+    const CUtensorMap* mk = is_retr ? &maps.rk : &maps.sk;
+    const CUtensorMap* mv = is_retr ? &maps.rv : &maps.sv;
+
+    if (tid == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(bar(bKFull + s), 1);
+            mbar_init(bar(bVFull + s), 1);
+            mbar_init(bar(bKEmpty + s), 1);
+            mbar_init(bar(bVEmpty + s), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(bSFull + s), 1);
+            mbar_init(bar(bPFull + s), 4);
+            mbar_init(bar(bPEmpty + s), 1);
+        }
+        mbar_init(bar(bODone), 1);
+        mbar_init(bar(bOFinal), 1);
+        mbar_init(bar(bDrain), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(base + kOffMisc, kTcTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        tma_prefetch_desc(mk);
+        tma_prefetch_desc(mv);
+    }
+    grid_dependency_wait();  // launched with programmatic stream serialization
+    grid_launch_dependents();
+
+    // The owner writes the new token into its slot first; its tile reads it back
+    // through TMA (generic-proxy stores made visible to the async proxy).
+    if (owns_new && warp == 4) {
+        const bf16* knew = p.k_new + (static_cast<int64_t>(b) * p.Hkv + g) * D;
+        const bf16* vnew = p.v_new + (static_cast<int64_t>(b) * p.Hkv + g) * D;
+        const int64_t slots = is_retr ? p.max_len : p.W;
+        const int64_t off = (static_cast<int64_t>(zrow) * slots + new_slot) * D;
+        bf16* dk = is_retr ? p.pools.rk : p.pools.sk;
+        bf16* dv = is_retr ? p.pools.rv : p.pools.sv;
+        if (lane < 16) {
+            *reinterpret_cast<uint4*>(dk + off + lane * 8) = ld_nc_v4(knew + lane * 8);
+        } else {
+            *reinterpret_cast<uint4*>(dv + off + (lane - 16) * 8) = ld_nc_v4(vnew + (lane - 16) * 8);
+        }
+        fence_proxy_async_global();
+    }
+    // Queries of the group as the B operand (rows G..15 zero).
+    for (int i = tid; i < kTcN * D / 8; i += kTcThreads) {
+        const int row = i / (D / 8);
+        const int c8 = (i % (D / 8)) * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (row < G) v = ld_nc_v4(p.q + (static_cast<int64_t>(b) * p.Hq + g * G + row) * D + c8);
+        *reinterpret_cast<uint4*>(sb + kOffQ + sw128_off16(row, c8)) = v;
+    }
+    // P buffers: rows G..15 stay zero.
+    for (int i = tid; i < 2 * kTcPBytes / 16; i += kTcThreads)
+        reinterpret_cast<uint4*>(sb + kOffP)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0 && n_tiles > 0) {
+            int issued = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int st = j % kTcStages;
+                const int row0 = static_cast<int>(r0) + j * kTcKeys;
+                if (j >= kTcStages) {
+                    const uint32_t par = ((j / kTcStages) - 1) & 1;
+                    if (!mbar_wait(bar(bKEmpty + st), par, abort_flag) ||
+                        !mbar_wait(bar(bVEmpty + st), par, abort_flag)) {
+                        tc_abort(p.err, abort_flag);
+                        break;
+                    }
+                }
+                mbar_arrive_expect_tx(bar(bKFull + st), kTcTile);
+                mbar_arrive_expect_tx(bar(bVFull + st), kTcTile);
+                for (int kb = 0; kb < D / 64; ++kb) {
+                    tma_load_3d(base + kOffK + st * kTcTile + kb * kTcColBlock, mk, bar(bKFull + st), kb * 64, row0,
+                                zrow);
+                    tma_load_3d(base + kOffV + st * kTcTile + kb * kTcColBlock, mv, bar(bVFull + st), kb * 64, row0,
+                                zrow);
+                }
+                issued = j + 1;
+            }
+            // Let every load this thread issued land before the CTA can exit.
+            for (int j = (issued > kTcStages ? issued - kTcStages : 0); j < issued; ++j) {
+                mbar_wait(bar(bKFull + j % kTcStages), (j / kTcStages) & 1, nullptr);
+                mbar_wait(bar(bVFull + j % kTcStages), (j / kTcStages) & 1, nullptr);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && n_tiles > 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kTcN, 0, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, kTcN, 1, 0);
+            // S^T(j) = K(j) Q^T into S buffer j&1.
+            auto qk = [&](int j) -> bool {
+                const int st = j % kTcStages;
+                if (!mbar_wait(bar(bKFull + st), (j / kTcStages) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t kt = base + kOffK + st * kTcTile;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t a = smem_desc_sw128(kt + (kk >> 2) * kTcColBlock + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bq = smem_desc_sw128(base + kOffQ + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+                    tc_mma_ss(tmem + (j & 1) * kTcN, a, bq, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar(bSFull + (j & 1)));
+                tc_commit(bar(bKEmpty + st));
+                return true;
+            };
+            bool ok = true;
+            for (int j = 0; ok && j < 2 && j < n_tiles; ++j) ok = qk(j);
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                const int st = j % kTcStages;
+                const int pb = j & 1;
+                if (!mbar_wait(bar(bVFull + st), (j / kTcStages) & 1, abort_flag) ||
+                    !mbar_wait(bar(bPFull + pb), (j >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t vt = base + kOffV + st * kTcTile;
+#pragma unroll
+                for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+                    // A = V^T: the V tile read MN-major (16 keys per step, two 64-column blocks)
+                    const uint64_t a = smem_desc_sw128(vt + kk * 2048, kTcColBlock, 1024);
+                    const uint64_t bp =
+                        smem_desc_sw128(base + kOffP + pb * kTcPBytes + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
+                    tc_mma_ss(tmem + kTcTmemO, a, bp, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(bar(bODone));
+                tc_commit(bar(bPEmpty + pb));
+                tc_commit(bar(bVEmpty + st));
+                if (j + 1 == n_tiles) tc_commit(bar(bOFinal));
+                if (j + 2 < n_tiles) ok = qk(j + 2);
+            }
+            if (!ok) tc_abort(p.err, abort_flag);
+            // Drain: every MMA issued above completes before TMEM is released.
+            tc_commit(bar(bDrain));
+            mbar_wait(bar(bDrain), 0, nullptr);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax: thread = key
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        float m[G], l[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            m[h] = -INFINITY;
+            l[h] = 0.f;
+        }
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int sbuf = j & 1;
+            if (!(ok && __all_sync(0xffffffffu, mbar_wait(bar(bSFull + sbuf), (j >> 1) & 1, abort_flag)))) ok = false;
+            float x[G];
+            if (ok) {
+                tc_fence_after();
+                uint32_t r[16];
+                tmem_ld16(tmem + lane_base + sbuf * kTcN, r);
+                tc_wait_ld();
+                const int64_t key = r0 + static_cast<int64_t>(j) * kTcKeys + tid;
+                const bool valid = key < r_end;
+#pragma unroll
+                for (int h = 0; h < G; ++h) x[h] = valid ? __uint_as_float(r[h]) * p.scale_log2 : -INFINITY;
+            } else {
+#pragma unroll
+                for (int h = 0; h < G; ++h) x[h] = -INFINITY;
+            }
+            // Raise the running maxima (and rescale O^T and l) only when a score
+            // exceeds them by more than 2^8; every thread takes the same decision.
+            bool need = false;
+#pragma unroll
+            for (int h = 0; h < G; ++h) need = need || (x[h] > m[h] + kTcRescale);
+            if (softmax_any(need)) {
+                volatile float* rr = red + (j & 1) * 4 * kTcN;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    float v = x[h];
+#pragma unroll
+                    for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                    if (lane == 0) rr[warp * kTcN + h] = v;
+                }
+                softmax_sync();
+                float factor[G];
+                bool any_factor = false;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float tmax = fmaxf(fmaxf(rr[h], rr[kTcN + h]), fmaxf(rr[2 * kTcN + h], rr[3 * kTcN + h]));
+                    factor[h] = 1.f;
+                    if (tmax > m[h]) {
+                        factor[h] = (m[h] == -INFINITY) ? 0.f : fast_exp2(m[h] - tmax);
+                        m[h] = tmax;
+                    }
+                    l[h] *= factor[h];
+                    any_factor = any_factor || factor[h] != 1.f;
+                }
+                // O^T rows are output columns: thread t rescales column t of every head,
+                // after PV(j-1) has written it (S(j) ready means PV(j-2) is complete, so
+                // the barrier's phase for PV(j-1) is the only one outstanding).
+                if (j >= 1 && __any_sync(0xffffffffu, any_factor)) {
+                    if (__all_sync(0xffffffffu, ok && mbar_wait(bar(bODone), (j - 1) & 1, abort_flag))) {
+                        tc_fence_after();
+                        uint32_t r[16];
+                        tmem_ld16(tmem + lane_base + kTcTmemO, r);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int h = 0; h < G; ++h) r[h] = __float_as_uint(__uint_as_float(r[h]) * factor[h]);
+                        tmem_st16(tmem + lane_base + kTcTmemO, r);
+                        tc_wait_st();
+                    } else {
+                        ok = false;
+                    }
+                }
+            }
+            // P^T(j): this thread's key column of every head.
+            const int pb = j & 1;
+            if (j >= 2 && !__all_sync(0xffffffffu, ok && mbar_wait(bar(bPEmpty + pb), ((j >> 1) - 1) & 1, abort_flag)))
+                ok = false;
+            if (ok) {
+                uint8_t* pbuf = sb + kOffP + pb * kTcPBytes;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float pv = (x[h] == -INFINITY) ? 0.f : fast_exp2(x[h] - m[h]);
+                    l[h] += pv;
+                    *reinterpret_cast<bf16*>(pbuf + sw128_off16(h, tid)) = __float2bfloat16_rn(pv);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(bPFull + pb));
+            }
+        }
+        // Row sums over the CTA's keys, then this thread's output column.
+        {
+            volatile float* rr = red;  // reused: [4 warps][16]
+            softmax_sync();
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float v = l[h];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0) rr[warp * kTcN + h] = v;
+            }
+            softmax_sync();
+#pragma unroll
+            for (int h = 0; h < G; ++h) l[h] = rr[h] + rr[kTcN + h] + rr[2 * kTcN + h] + rr[3 * kTcN + h];
+        }
+        const int64_t item = (static_cast<int64_t>(b) * p.n_retr + ri) * p.nsplit + split;
+        const bool final_now = !is_retr || p.nsplit == 1;
+        if (n_tiles > 0 && __all_sync(0xffffffffu, ok && mbar_wait(bar(bOFinal), 0, abort_flag))) {
+            tc_fence_after();
+            uint32_t r[16];
+            tmem_ld16(tmem + lane_base + kTcTmemO, r);
+            tc_wait_ld();
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float o = l[h] > 0.f ? __uint_as_float(r[h]) / l[h] : 0.f;
+                if (final_now) {
+                    p.out[(static_cast<int64_t>(b) * p.Hq + g * G + h) * D + tid] = __float2bfloat16_rn(o);
+                } else {
+                    p.part_o[(item * G + h) * D + tid] = o;
+                    if (tid == 0) p.part_lse[item * G + h] = l[h] > 0.f ? m[h] + __log2f(l[h]) : -INFINITY;
+                }
+            }
+        } else {
+            // a split without rows (ragged batch), or an abort: an empty partial
+            if (n_tiles > 0) tc_abort(p.err, abort_flag);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                if (!final_now) {
+                    p.part_o[(item * G + h) * D + tid] = 0.f;
+                    if (tid == 0) p.part_lse[item * G + h] = -INFINITY;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) tmem_dealloc(tmem, kTcTmemCols);
+    if (!is_retr || p.nsplit == 1) return;
+
+    // Split-KV merge (D4): the last CTA of this (b, KV head) combines the
+    // partials, thread t column t of every head.
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const uint32_t prev = atomicAdd(&p.counters[b * p.Hkv + g], 1u);
+        *last_flag = (prev == static_cast<uint32_t>(p.nsplit - 1));
+    }
+    __syncthreads();
+    if (!*last_flag) return;
+    __threadfence();
+    if (tid < D) {
+        const int64_t item0 = (static_cast<int64_t>(b) * p.n_retr + ri) * p.nsplit;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float M = -INFINITY, Ls = 0.f, acc = 0.f;
+#pragma unroll 4
+            for (int s = 0; s < p.nsplit; ++s) {
+                const float x = __ldcg(p.part_lse + (item0 + s) * G + h);
+                const float o = __ldcg(p.part_o + ((item0 + s) * G + h) * D + tid);
+                if (x > M) {
+                    const float f = fast_exp2(M - x);  // 0 while M is -inf
+                    Ls *= f;
+                    acc *= f;
+                    M = x;
+                }
+                const float w = (x == -INFINITY) ? 0.f : fast_exp2(x - M);
+                Ls += w;
+                acc = fmaf(w, o, acc);
+            }
+            p.out[(static_cast<int64_t>(b) * p.Hq + g * G + h) * D + tid] = __float2bfloat16_rn(acc / Ls);
+        }
+    }
+    if (tid == 0) p.counters[b * p.Hkv + g] = 0u;  // ready for the next step (stream-ordered)
+}
+
+template <int G>
+cudaError_t launch_tc_g(const DecodeParams& p, const DecodeMaps& maps, unsigned grid, cudaStream_t s) {
+    static SmemLimitOnce limit;
+    const cudaError_t e = limit.apply(reinterpret_cast<const void*>(&decode_tc_kernel<G>), kTcSmem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = kTcSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_tc_kernel<G>, p, maps);
+}
+
+}  // namespace
+
+cudaError_t launch_decode_tc(const DecodeParams& p, const DecodeMaps& maps, cudaStream_t s) {
+    const unsigned grid = static_cast<unsigned>(p.B * p.n_retr * p.nsplit + p.B * p.n_strm);
+    if (grid == 0) return cudaSuccess;
+    if (!decode_on_tensor_cores(p.G, p.D, p.fp8 != 0)) return cudaErrorInvalidValue;
+    if (p.G == 4) return launch_tc_g<4>(p, maps, grid, s);
+    if (p.G == 8) return launch_tc_g<8>(p, maps, grid, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace duo

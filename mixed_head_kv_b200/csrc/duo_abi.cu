@@ -567,7 +567,7 @@ duo_status duo_decode(duo_cache* c, int32_t layer, const void* q, const void* k_
     const int64_t nsplit = decode_plan(c, layer, rows);
     p.split_rows = (rows + nsplit - 1) / nsplit;
     p.nsplit = static_cast<int32_t>((rows + p.split_rows - 1) / p.split_rows);
-    if (launch_decode(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUO_ERR_CUDA;
+    if (launch_decode(p, decode_maps(c), static_cast<cudaStream_t>(stream)) != cudaSuccess) return DUO_ERR_CUDA;
     int64_t* L = seq_lens(c, layer);
     for (int32_t b = 0; b < c->lay.batch; ++b) L[b] += 1;
     return DUO_OK;

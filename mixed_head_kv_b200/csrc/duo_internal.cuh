@@ -95,6 +95,15 @@ constexpr int kDecodeThreads = 128;
 // and register budget are sized for it).
 __host__ __device__ constexpr int decode_ctas_per_sm(int G) { return (G == 2 || G == 4) ? 3 : 2; }
 
+// Query groups of 4 and 8 heads over bf16 caches with head_dim 128 decode on the
+// tensor cores (decode_tc.cu, one CTA per SM); everything else on the CUDA cores.
+__host__ __device__ constexpr bool decode_on_tensor_cores(int G, int D, bool fp8) {
+    return (G == 4 || G == 8) && D == 128 && !fp8;
+}
+__host__ __device__ constexpr int decode_slots_per_sm(int G, int D, bool fp8) {
+    return decode_on_tensor_cores(G, D, fp8) ? 1 : decode_ctas_per_sm(G);
+}
+
 // Splits per retrieval (b, KV head) for one decode step. Every CTA streams
 // its rows at about the same rate, so the step takes about
 //   waves * (rows of the longest CTA + a fixed per-CTA cost),
@@ -102,12 +111,12 @@ __host__ __device__ constexpr int decode_ctas_per_sm(int G) { return (G == 2 || 
 // sink + recent rows each. Pick the split count (>= 256 rows per split, at most
 // kDecodeMaxSplits) that minimises that estimate.
 inline int64_t plan_decode_splits(int64_t batch, int64_t n_retr, int64_t n_strm, int64_t rows, int64_t strm_rows,
-                                  int num_sms, int G) {
+                                  int num_sms, int G, int D, bool fp8) {
     if (n_retr <= 0) return 1;
     constexpr int64_t kCtaCostRows = 64;
     const int64_t pairs = batch * n_retr;
     const int64_t strm_items = batch * n_strm;
-    const int64_t slots = static_cast<int64_t>(num_sms) * decode_ctas_per_sm(G);
+    const int64_t slots = static_cast<int64_t>(num_sms) * decode_slots_per_sm(G, D, fp8);
     int64_t max_split = (rows + 255) / 256;
     if (max_split > kDecodeMaxSplits) max_split = kDecodeMaxSplits;
     if (max_split < 1) max_split = 1;
@@ -154,7 +163,14 @@ struct DecodeParams {
     uint64_t test_timeout_ns;           // the withheld copy's wait limit
     int64_t seq_len[kMaxRaggedBatch];   // tokens cached before this step, per sequence
 };
-cudaError_t launch_decode(const DecodeParams& p, cudaStream_t s);
+// TMA maps of the cache pools (box 64 x 128 rows), for the tensor-core decode.
+struct DecodeMaps {
+    CUtensorMap rk, rv, sk, sv;
+};
+// One decode step: on the tensor cores when decode_on_tensor_cores() (and no
+// test of the bounded waits is armed), else on the CUDA cores.
+cudaError_t launch_decode(const DecodeParams& p, const DecodeMaps& maps, cudaStream_t s);
+cudaError_t launch_decode_tc(const DecodeParams& p, const DecodeMaps& maps, cudaStream_t s);
 
 // ------------------------------------------------------------------ prefill
 constexpr int kTileQ = 128;   // query rows per CTA (one TMEM lane each)
@@ -219,6 +235,9 @@ struct duo_cache {
     std::vector<int64_t> plan_nsplit;            // [layers] the plan's split count
 };
 
+// The pool tensor maps of a cache, as the decode launch takes them.
+inline duo::DecodeMaps decode_maps(const duo_cache* c) { return duo::DecodeMaps{c->map_rk, c->map_rv, c->map_sk, c->map_sv}; }
+
 // Per-sequence lengths of one layer ([batch] host values).
 inline int64_t* seq_lens(duo_cache* c, int32_t layer) {
     return c->len.data() + static_cast<size_t>(layer) * c->lay.batch;
@@ -263,7 +282,7 @@ inline int64_t decode_plan(duo_cache* c, int32_t layer, int64_t rows) {
         const duo::DecodeParams& t = c->decode_tmpl[layer];
         c->plan_nsplit[layer] =
             duo::plan_decode_splits(c->lay.batch, t.n_retr, t.n_strm, rows, rows < c->W ? rows : c->W, c->num_sms,
-                                    c->G);
+                                    c->G, c->lay.head_dim, c->fp8);
         c->plan_key[layer] = key;
     }
     return c->plan_nsplit[layer];

@@ -8,8 +8,9 @@ of the library instead. These tests run it through the C ABI next to
 duo_decode on identical caches, for two calls in a row, and require
   - the fp64 oracle's outputs within the tolerance of the other parity tests,
   - duo_decode's outputs within the same tolerance,
-on uniform, GQA (G = 8) and ragged batches, and on a batch whose full split
-plan does not fit the array (fewer, longer splits are used then).
+on uniform, GQA (G = 8) and ragged batches, and on batches whose full split
+plan does not fit the array (fewer, longer splits are used then), on both the
+tensor-core and the CUDA-core decode kernels.
 
 This file is collected last on purpose and also passes when run on its own.
 """
@@ -121,10 +122,13 @@ def test_static_scratch_ragged_batch(duo):
     assert static_cache.error_flags() == 0
 
 
-def _planned_splits(batch, n_retr, n_strm, rows, strm_rows, num_sms, G):
+def _planned_splits(batch, n_retr, n_strm, rows, strm_rows, num_sms, G, D):
     """The split count duo_decode would pick (restated here only to check that the
-    shape below really exceeds the static array; the library's own plan decides)."""
-    slots = num_sms * (3 if G in (2, 4) else 2)
+    shapes below really exceed the static array; the library's own plan decides).
+    Query groups of 4 and 8 with head_dim 128 run one tensor-core CTA per SM; the
+    CUDA-core kernel runs 3 CTAs per SM for groups of 2 and 4, 2 otherwise."""
+    per_sm = 1 if (G in (4, 8) and D == 128) else (3 if G in (2, 4) else 2)
+    slots = num_sms * per_sm
     best, best_cost = 1, None
     for ns in range(1, min(256, max(1, (rows + 255) // 256)) + 1):
         waves = (batch * n_retr * ns + batch * n_strm + slots - 1) // slots
@@ -135,20 +139,26 @@ def _planned_splits(batch, n_retr, n_strm, rows, strm_rows, num_sms, G):
     return best
 
 
-def test_static_scratch_clamps_splits_to_the_array(duo):
-    """32 sequences x 3 retrieval KV heads x G = 8 at 16K context: the full split
-    plan needs more partials than the array holds, so the call serves the step
-    with fewer, longer splits; outputs still match the oracle and duo_decode."""
-    shape = dict(batch=32, num_q_heads=128, num_kv_heads=16, head_dim=128, sink=64, recent=256,
-                 mask=(1, 0, 0, 0, 0, 1, 0, 0, 0, 0, 1, 0, 0, 0, 0, 0))
+@pytest.mark.parametrize("shape", [
+    # tensor-core decode: 64 sequences x 4 retrieval KV heads x G = 8, head_dim 128, 8K context
+    dict(batch=64, num_q_heads=128, num_kv_heads=16, head_dim=128, L=8192, retr=(0, 3, 5, 12)),
+    # CUDA-core decode: 64 sequences x 3 retrieval KV heads x G = 8, head_dim 64, 16K context
+    dict(batch=64, num_q_heads=256, num_kv_heads=32, head_dim=64, L=16384, retr=(1, 9, 30)),
+], ids=["tensor_core_path", "cuda_core_path"])
+def test_static_scratch_clamps_splits_to_the_array(duo, shape):
+    """The full split plan needs more partials than the array holds, so the call
+    serves the step with fewer, longer splits; outputs still match the oracle and
+    duo_decode."""
+    mask = tuple(1 if g in shape["retr"] else 0 for g in range(shape["num_kv_heads"]))
+    shape = dict(shape, sink=64, recent=256, mask=mask)
     w = _workload(shape, seed=11)
-    L = 16384
+    L = shape["L"]
     G, D = w.group, w.head_dim
-    n_retr = sum(shape["mask"])
+    n_retr = sum(mask)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     counters = (w.batch * w.num_kv_heads * 4 + 255) // 256 * 256
     fit = (duo.DUO_STATIC_SCRATCH_BYTES - counters - 256) // (w.batch * n_retr * G * (D + 1) * 4)
-    planned = _planned_splits(w.batch, n_retr, w.num_kv_heads - n_retr, L + 1, w.sink + w.recent, sms, G)
+    planned = _planned_splits(w.batch, n_retr, w.num_kv_heads - n_retr, L + 1, w.sink + w.recent, sms, G, D)
     assert 1 <= fit < planned, (fit, planned)  # the premise: the plan does not fit the array
     ref_cache, static_cache = _caches(duo, w, L + 8)
     for c0 in range(0, L, 4096):
@@ -156,7 +166,7 @@ def test_static_scratch_clamps_splits_to_the_array(duo):
         for c in (ref_cache, static_cache):
             c.append(0, kk, vv)
     q, k, v = workloads.tokens(w, 0, L, 2, device="cuda")
-    sampled = (0, 17, 31)
+    sampled = (0, 17, w.batch - 1)
     kh, vh = workloads.tokens(w, 0, 0, L, device="cuda", which="kv")
     hist = [torch.cat([h, x], dim=1)[list(sampled)].cpu() for h, x in ((kh, k), (vh, v))]
     del kh, vh
@@ -167,7 +177,7 @@ def test_static_scratch_clamps_splits_to_the_array(duo):
         for i, b in enumerate(sampled):
             ref = oracle.attention(q[b:b + 1, step:step + 1].cpu().permute(0, 2, 1, 3), np.array([p]),
                                    hist[0][i:i + 1, :p + 1].permute(0, 2, 1, 3),
-                                   hist[1][i:i + 1, :p + 1].permute(0, 2, 1, 3), shape["mask"], w.sink, w.recent)
+                                   hist[1][i:i + 1, :p + 1].permute(0, 2, 1, 3), mask, w.sink, w.recent)
             assert_close(rb[b], ref[0, :, 0], f"step {step} seq {b} vs oracle")
     assert static_cache.error_flags() == 0
 
