@@ -608,73 +608,76 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
     if (!*sm_last) return;
     __threadfence();
     // The partials of this (b, KV head) are contiguous: [nsplit][G][D] floats and
-    // [nsplit][G] log-sum-exps. One coalesced float4 pass: each thread folds an
-    // independent subset of the splits with a running max (the log-sum-exp and
-    // the partial of a split are loaded together), then the subsets are combined.
+    // [nsplit][G] log-sum-exps. First every split's weight per head, from one
+    // coalesced load of the log-sum-exps: w = 2^(lse - max) / sum over the splits
+    // (a split without rows, lse = -inf, weighs 0). Then each thread sums its
+    // float4 unit over a subset of the splits, its loads independent of each
+    // other, and the subsets are added.
     const int64_t item0 = (static_cast<int64_t>(b) * p.n_retr + ri) * p.nsplit;
     const int ns = p.nsplit;
     constexpr int kUnits = G * D / 4;  // float4 units of one split's partial
     constexpr int kRep = kUnits >= kDecodeThreads ? 1 : kDecodeThreads / kUnits;
-    float4* sm_acc = reinterpret_cast<float4*>(smem);                 // [kRep][kUnits]
-    float* sm_mx = reinterpret_cast<float*>(sm_acc + kRep * kUnits);  // [kRep][kUnits]
-    float* sm_ls = sm_mx + kRep * kUnits;                             // [kRep][kUnits]
+    float4* sm_acc = reinterpret_cast<float4*>(smem);                  // [kRep][kUnits]
+    float* sm_w = reinterpret_cast<float*>(sm_acc + kRep * kUnits);    // [ns][G] log-sum-exps, then weights
+    float* sm_norm = sm_w + kDecodeMaxSplits * G;                      // [G] max, [G] 1 / sum
     const float4* po = reinterpret_cast<const float4*>(p.part_o + item0 * G * D);
     const float* pl = p.part_lse + item0 * G;
     __syncthreads();  // the per-warp merge arrays above are no longer read
+    for (int i = tid; i < ns * G; i += kDecodeThreads) sm_w[i] = __ldcg(pl + i);
+    __syncthreads();
+    for (int h = warp; h < G; h += kWarps) {
+        float M = -INFINITY;
+        for (int sp = lane; sp < ns; sp += 32) M = fmaxf(M, sm_w[sp * G + h]);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float S = 0.f;
+        for (int sp = lane; sp < ns; sp += 32) {
+            const float x = sm_w[sp * G + h];
+            S += (x == -INFINITY) ? 0.f : fast_exp2(x - M);
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) S += __shfl_xor_sync(0xffffffffu, S, off);
+        if (lane == 0) {
+            sm_norm[h] = M;
+            sm_norm[G + h] = 1.f / S;  // S >= 1: the split holding the maximum weighs 1
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < ns * G; i += kDecodeThreads) {
+        const int h = i % G;
+        const float x = sm_w[i];
+        sm_w[i] = (x == -INFINITY) ? 0.f : fast_exp2(x - sm_norm[h]) * sm_norm[G + h];
+    }
+    __syncthreads();
     for (int u = tid % kUnits; u < kUnits; u += kDecodeThreads) {
         const int h = (u * 4) / D;
         const int rep = tid / kUnits;  // < kRep
-        float M = -INFINITY, Ls = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int s = rep; s < ns; s += kRep) {
-            const float x = __ldcg(pl + static_cast<int64_t>(s) * G + h);
-            const float4 o = __ldcg(po + static_cast<int64_t>(s) * kUnits + u);
-            if (x > M) {
-                const float f = fast_exp2(M - x);  // 0 while M is -inf
-                Ls *= f;
-                acc.x *= f;
-                acc.y *= f;
-                acc.z *= f;
-                acc.w *= f;
-                M = x;
-            }
-            // A split without rows (ragged batch) has lse = -inf and weight 0; a select,
-            // not a branch, keeps the loads of the unrolled iterations together.
-            const float w = (x == -INFINITY) ? 0.f : fast_exp2(x - M);
-            Ls += w;
+#pragma unroll 8
+        for (int sp = rep; sp < ns; sp += kRep) {
+            const float w = sm_w[sp * G + h];
+            const float4 o = __ldcg(po + static_cast<int64_t>(sp) * kUnits + u);
             acc.x = fmaf(w, o.x, acc.x);
             acc.y = fmaf(w, o.y, acc.y);
             acc.z = fmaf(w, o.z, acc.z);
             acc.w = fmaf(w, o.w, acc.w);
         }
         sm_acc[rep * kUnits + u] = acc;
-        sm_mx[rep * kUnits + u] = M;
-        sm_ls[rep * kUnits + u] = Ls;
     }
     __syncthreads();
     for (int u = tid; u < kUnits; u += kDecodeThreads) {
-        float M = -INFINITY;
-        for (int r = 0; r < kRep; ++r) M = fmaxf(M, sm_mx[r * kUnits + u]);
-        float Ls = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int r = 0; r < kRep; ++r) {
-            const float mr = sm_mx[r * kUnits + u];
-            if (mr == -INFINITY) continue;  // this subset held no split
-            const float f = fast_exp2(mr - M);
+        float4 acc = sm_acc[u];
+        for (int r = 1; r < kRep; ++r) {
             const float4 x = sm_acc[r * kUnits + u];
-            Ls = fmaf(f, sm_ls[r * kUnits + u], Ls);
-            acc.x = fmaf(f, x.x, acc.x);
-            acc.y = fmaf(f, x.y, acc.y);
-            acc.z = fmaf(f, x.z, acc.z);
-            acc.w = fmaf(f, x.w, acc.w);
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
         }
-        const float inv = 1.f / Ls;
         const int h = (u * 4) / D;
         const int d = (u * 4) % D;
         bf16* o = p.out + (static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d;
-        *reinterpret_cast<uint2*>(o) =
-            make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+        *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
     }
     if (tid == 0) p.counters[b * p.Hkv + g] = 0u;  // ready for the next step (stream-ordered)
 }
@@ -694,7 +697,8 @@ template <int D, int G, bool Fp8>
 cudaError_t launch_dg(const DecodeParams& p, unsigned grid, cudaStream_t s) {
     constexpr int smem = Geom<D, G>::kSmem;
     static_assert((kWarps * 2 * G + kWarps * G * D) * 4 <= Geom<D, G>::kRingBytes, "warp merge arrays fit in the ring");
-    static_assert((16 + 8) * (G * D / 4 >= kDecodeThreads ? G * D / 4 : kDecodeThreads) <= Geom<D, G>::kRingBytes,
+    static_assert(16 * (G * D / 4 >= kDecodeThreads ? G * D / 4 : kDecodeThreads) + 4 * (kDecodeMaxSplits + 2) * G <=
+                      Geom<D, G>::kRingBytes,
                   "split merge arrays fit in the ring");
     static SmemLimitOnce limit;
     static_assert(decode_ctas_per_sm(G) == 2 || decode_ctas_per_sm(G) == 3, "one of the two kernels");

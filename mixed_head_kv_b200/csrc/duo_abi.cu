@@ -105,6 +105,21 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, 
     return r == CUDA_SUCCESS;
 }
 
+// One-byte-code pool map for E4M3 retrieval caches: (D, slots, heads*B) uint8,
+// box (D, 128, 1), no swizzle (the decode converts the codes itself).
+bool make_code_pool_map(CUtensorMap* m, const void* base, int64_t D, int64_t slots, int64_t zdim) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t d[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(slots),
+                             static_cast<cuuint64_t>(zdim < 1 ? 1 : zdim)};
+    const cuuint64_t st[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(D * slots)};
+    const cuuint32_t b[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(kTileK), 1};
+    const cuuint32_t e[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), d, st, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Pool map: (D, slots, heads*B), box (64, 128, 1).
 bool make_pool_map(CUtensorMap* m, const void* base, int64_t D, int64_t slots, int64_t zdim) {
     const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(slots),
@@ -228,6 +243,12 @@ duo_status duo_cache_alloc(const duo_layout* layout, const uint8_t* is_retrieval
     if (any_bf16 &&
         (!make_pool_map(&c->map_rk, rk, D, rslots, rz) || !make_pool_map(&c->map_rv, rv, D, rslots, rz) ||
          !make_pool_map(&c->map_sk, sk, D, sslots, sz) || !make_pool_map(&c->map_sv, sv, D, sslots, sz))) {
+        delete c;
+        return DUO_ERR_CUDA;
+    }
+    if (c->fp8 && nr > 0 &&
+        (!make_code_pool_map(&c->map_rk8, c->pools.rk, D, L.max_len, static_cast<int64_t>(nr) * L.batch) ||
+         !make_code_pool_map(&c->map_rv8, c->pools.rv, D, L.max_len, static_cast<int64_t>(nr) * L.batch))) {
         delete c;
         return DUO_ERR_CUDA;
     }

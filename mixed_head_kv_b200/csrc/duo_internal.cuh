@@ -95,10 +95,11 @@ constexpr int kDecodeThreads = 128;
 // and register budget are sized for it).
 __host__ __device__ constexpr int decode_ctas_per_sm(int G) { return (G == 2 || G == 4) ? 3 : 2; }
 
-// Query groups of 4 and 8 heads over bf16 caches with head_dim 128 decode on the
-// tensor cores (decode_tc.cu, one CTA per SM); everything else on the CUDA cores.
-__host__ __device__ constexpr bool decode_on_tensor_cores(int G, int D, bool fp8) {
-    return (G == 4 || G == 8) && D == 128 && !fp8;
+// Query groups of 4 and 8 heads with head_dim 128 decode on the tensor cores
+// (decode_tc.cu, one CTA per SM; E4M3 retrieval rows are converted to f16 in
+// shared memory); everything else on the CUDA cores.
+__host__ __device__ constexpr bool decode_on_tensor_cores(int G, int D, bool /*fp8*/) {
+    return (G == 4 || G == 8) && D == 128;
 }
 __host__ __device__ constexpr int decode_slots_per_sm(int G, int D, bool fp8) {
     return decode_on_tensor_cores(G, D, fp8) ? 1 : decode_ctas_per_sm(G);
@@ -163,9 +164,12 @@ struct DecodeParams {
     uint64_t test_timeout_ns;           // the withheld copy's wait limit
     int64_t seq_len[kMaxRaggedBatch];   // tokens cached before this step, per sequence
 };
-// TMA maps of the cache pools (box 64 x 128 rows), for the tensor-core decode.
+// TMA maps of the cache pools, for the tensor-core decode: bf16 pools with box
+// 64 x 128 rows (128-byte swizzle); for E4M3 caches also the retrieval pools as
+// one-byte codes with box D x 128 rows (no swizzle).
 struct DecodeMaps {
     CUtensorMap rk, rv, sk, sv;
+    CUtensorMap rk8, rv8;
 };
 // One decode step: on the tensor cores when decode_on_tensor_cores() (and no
 // test of the bounded waits is armed), else on the CUDA cores.
@@ -225,6 +229,7 @@ struct duo_cache {
     uint32_t* counters = nullptr;
     uint32_t* err = nullptr;
     CUtensorMap map_rk{}, map_rv{}, map_sk{}, map_sv{};
+    CUtensorMap map_rk8{}, map_rv8{};   // E4M3 caches: the retrieval pools as one-byte codes
     int32_t test_wait = 0;              // duo_cache_test_wait_timeout: launch kinds still to withhold a copy
     uint64_t test_wait_ns = 0;
     bool fp8 = false;                   // retrieval pools hold E4M3 codes
@@ -236,7 +241,9 @@ struct duo_cache {
 };
 
 // The pool tensor maps of a cache, as the decode launch takes them.
-inline duo::DecodeMaps decode_maps(const duo_cache* c) { return duo::DecodeMaps{c->map_rk, c->map_rv, c->map_sk, c->map_sv}; }
+inline duo::DecodeMaps decode_maps(const duo_cache* c) {
+    return duo::DecodeMaps{c->map_rk, c->map_rv, c->map_sk, c->map_sv, c->map_rk8, c->map_rv8};
+}
 
 // Per-sequence lengths of one layer ([batch] host values).
 inline int64_t* seq_lens(duo_cache* c, int32_t layer) {

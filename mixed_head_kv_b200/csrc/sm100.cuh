@@ -223,6 +223,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
            | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// Instruction descriptor of kind::f16 with f16 A/B and fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4)                                  // D format: f32
+           | (static_cast<uint32_t>(a_mn) << 15)      // A major (A, B format 0: f16)
+           | (static_cast<uint32_t>(b_mn) << 16)      // B major
+           | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
 // ---------------------------------------------------------------- programmatic dependent launch
 // Block until the grids this launch depends on (earlier work in the stream)
 // have completed and their memory operations are visible.

@@ -36,8 +36,10 @@ def _inv(s):
     return float(np.float32(1.0) / np.float32(s))
 
 
-@pytest.mark.parametrize("G,D", [(1, 128), (4, 64)])
+@pytest.mark.parametrize("G,D", [(1, 128), (4, 64), (4, 128), (8, 128)])
 def test_fp8_append_codes_and_decode(duo, G, D):
+    """Groups of 4 and 8 with head_dim 128 run the tensor-core decode (codes
+    converted to f16 in shared memory); the others the CUDA-core kernel."""
     Hkv = 4
     w = make_workload(B=2, Hq=Hkv * G, Hkv=Hkv, D=D, S=4, R=64, mask=[1, 0, 1, 0])
     L, steps = 700, 4
@@ -116,11 +118,13 @@ def _fp8_ref(q_row, k_hist, v_hist, mask, G, w, k_scale, v_scale, p):
     return ref
 
 
+@pytest.mark.parametrize("G", [2, 4])
 @pytest.mark.parametrize("entry", ["duo_decode", "duo_decode_static_scratch"])
-def test_fp8_long_context_split_decode(duo, entry):
-    """20K cached tokens (many splits and the log-sum-exp merge), GQA G = 2, both
-    decode entry points; sink-like keys (x8) in the first positions."""
-    w = workloads.Workload("fp8_long", batch=1, num_q_heads=8, num_kv_heads=4, head_dim=128, sink=64, recent=256,
+def test_fp8_long_context_split_decode(duo, entry, G):
+    """20K cached tokens (many splits and the log-sum-exp merge), GQA G = 2 (CUDA
+    cores) and 4 (tensor cores), both decode entry points; sink-like keys (x8) in
+    the first positions."""
+    w = workloads.Workload("fp8_long", batch=1, num_q_heads=4 * G, num_kv_heads=4, head_dim=128, sink=64, recent=256,
                            retrieval_ratio=0.5, explicit_retrieval=(0, 1, 1, 0), seed=9, sink_key_scale=8)
     L, steps = 20000, 2
     k_scale, v_scale = [1.0, 0.125, 0.75, 1.0], [1.0, 0.5, 3.0, 1.0]
@@ -128,10 +132,10 @@ def test_fp8_long_context_split_decode(duo, entry):
     call = getattr(duo, entry)
     for t in range(steps):
         p = L + t
-        o = torch.full((1, 8, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+        o = torch.full((1, 4 * G, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
         assert call(cache.handle, 0, q[:, p].cuda(), k[:, p].cuda(), v[:, p].cuda(), o) == duo.DUO_OK
         torch.cuda.synchronize()
-        ref = _fp8_ref(q[:, p:p + 1], k[:, :p + 1], v[:, :p + 1], mask, 2, w, k_scale, v_scale, p)
+        ref = _fp8_ref(q[:, p:p + 1], k[:, :p + 1], v[:, :p + 1], mask, G, w, k_scale, v_scale, p)
         assert_close(o.cpu(), ref, f"{entry} step {t}")
     assert cache.error_flags() == 0
 

@@ -113,6 +113,54 @@ def test_llama3_gqa_decode_b4_128k(duo):
 SWEEP = [(r, 256) for r in (0.0, 0.25, 0.5, 0.75, 1.0)] + [(0.0, 1024), (0.25, 1024), (0.5, 1024)]
 
 
+def test_llama3_gqa_decode_b4_128k_e4m3(duo):
+    """The Llama-3-8B-shaped GQA decode (batch 4, 128K) over E4M3 retrieval caches
+    with per-head scales, in the benchmark's launch configuration (tensor-core
+    decode, codes converted to f16): every output against the oracle's attention
+    over the codes (streaming heads over bf16 rows), and the codes of a
+    retrieval head bit-exact against the oracle's quantizer."""
+    w = workloads.LLAMA3_GQA
+    mask = workloads.retrieval_mask(w)
+    L, steps, G = w.context, 2, w.group
+    ks = [0.5 + 0.25 * g for g in range(w.num_kv_heads)]
+    vs = [1.5 - 0.125 * g for g in range(w.num_kv_heads)]
+    cache = duo.DuoCache(1, w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.sink, w.recent, L + steps, mask,
+                         kv_format=duo.DUO_KV_E4M3)
+    cache.set_kv_scales(0, ks, vs)
+    for c0 in range(0, L, 16384):
+        kk, vv = workloads.tokens(w, 0, c0, 16384, device="cuda", which="kv")
+        cache.append(0, kk, vv)
+    q, k, v = workloads.tokens(w, 0, L, steps, device="cuda")
+    outs = []
+    for t in range(steps):
+        o = torch.full_like(q[:, t], float("nan"))
+        cache.decode(0, q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(), o)
+        outs.append(o)
+    torch.cuda.synchronize()
+    assert cache.error_flags() == 0
+    kh, vh = (x.cpu() for x in workloads.tokens(w, 0, 0, L + steps, device="cuda", which="kv"))
+    qc = q.cpu()
+    inv = lambda x: float(np.float32(1.0) / np.float32(x))
+    g0 = mask.index(1)
+    ck, cv, _ = cache.head_view(0, g0)
+    for b in range(w.batch):
+        assert np.array_equal(ck[b, :L + steps].cpu().numpy(), oracle.e4m3_quantize(kh[b, :, g0], inv(ks[g0])))
+        assert np.array_equal(cv[b, :L + steps].cpu().numpy(), oracle.e4m3_quantize(vh[b, :, g0], inv(vs[g0])))
+    scale = 1.0 / np.sqrt(w.head_dim)
+    for t in range(steps):
+        p = L + t
+        ref = _oracle_rows(w, qc[:, t:t + 1], np.array([p]), kh[:, :p + 1], vh[:, :p + 1], mask)[:, 0]
+        for g in range(w.num_kv_heads):
+            if not mask[g]:
+                continue
+            for b in range(w.batch):
+                kc = oracle.e4m3_quantize(kh[b, :p + 1, g], inv(ks[g]))
+                vc = oracle.e4m3_quantize(vh[b, :p + 1, g], inv(vs[g]))
+                for h in range(g * G, (g + 1) * G):
+                    ref[b, h], _ = oracle.attend_rows_e4m3(qc[b, t, h], kc, vc, ks[g], vs[g], scale)
+        assert_close(outs[t].cpu(), ref, f"e4m3 step {t}")
+
+
 @pytest.mark.parametrize("ratio,recent", SWEEP)
 def test_mha_sweep_decode_b8_64k(duo, ratio, recent):
     """MHA retrieval-ratio sweep: 32 heads, batch 8, 64K cached tokens."""
