@@ -19,7 +19,7 @@
 //   warp 4     TMA producer of the K and V tiles (3-stage rings, 128-B swizzle);
 //   warp 5     TMEM allocator and MMA issuer (one thread);
 //   warps 6-13 (E4M3 caches only) converters: a retrieval item's K and V tiles
-//              arrive as one-byte codes (2-stage staging rings, K and V apart)
+//              arrive as one-byte codes (staging rings of 3 K and 2 V stages)
 //              and these warps write them as f16 into 128-B-swizzled operand
 //              tiles (2 stages each): warps 6-9 the K tiles, warps 10-13 the V
 //              tiles, each group on its own chain (a K stage is free once its
@@ -68,9 +68,13 @@ struct TcLayout {
     static constexpr int kStages = Fp8 ? 2 : 3;  // operand stages (K and V tiles)
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kOffK + kStages * kTcTile;
-    static constexpr int kOffCK = kOffV + kStages * kTcTile;          // E4M3 code staging (2 stages)
-    static constexpr int kOffCV = kOffCK + (Fp8 ? 2 * kTcCodeTile : 0);
-    static constexpr int kOffQ = kOffCV + (Fp8 ? 2 * kTcCodeTile : 0);
+    // E4M3 code staging: 3 stages of K codes (their loads run two tiles ahead of
+    // the K conversion), 2 of V codes (the V conversion of tile j waits for PV(j-2)).
+    static constexpr int kCodeStagesK = 3;
+    static constexpr int kCodeStagesV = 2;
+    static constexpr int kOffCK = kOffV + kStages * kTcTile;
+    static constexpr int kOffCV = kOffCK + (Fp8 ? kCodeStagesK * kTcCodeTile : 0);
+    static constexpr int kOffQ = kOffCV + (Fp8 ? kCodeStagesV * kTcCodeTile : 0);
     static constexpr int kOffP = kOffQ + kTcQBytes;                 // 2 buffers
     static constexpr int kOffBar = kOffP + 2 * kTcPBytes;
     static constexpr int kOffRed = kOffBar + 40 * 8;                // [2][4 warps][16 heads] floats
@@ -90,10 +94,10 @@ constexpr int bPEmpty = 16;  // + P buffer
 constexpr int bODone = 18;   // one phase per tile
 constexpr int bOFinal = 19;
 constexpr int bDrain = 20;
-constexpr int bCKFull = 21;   // + staging stage: K codes loaded (E4M3)
-constexpr int bCVFull = 23;   // + staging stage: V codes loaded
-constexpr int bCKEmpty = 25;  // + staging stage: K codes converted (4 converter warps)
-constexpr int bCVEmpty = 27;  // + staging stage: V codes converted
+constexpr int bCKFull = 21;   // + K staging stage (3): K codes loaded (E4M3)
+constexpr int bCVFull = 24;   // + V staging stage (2): V codes loaded
+constexpr int bCKEmpty = 26;  // + K staging stage: K codes converted (4 converter warps)
+constexpr int bCVEmpty = 29;  // + V staging stage: V codes converted
 
 // TMEM columns: S^T buffers [0,16) [16,32), O^T [32,48)
 constexpr uint32_t kTcTmemCols = 64;
@@ -235,9 +239,13 @@ __global__ void __launch_bounds__(TcLayout<Fp8>::kThreads, 1)
             mbar_init(bar(bSFull + s), 1);
             mbar_init(bar(bPFull + s), 4);
             mbar_init(bar(bPEmpty + s), 1);
+        }
+        for (int s = 0; s < Lay::kCodeStagesK; ++s) {
             mbar_init(bar(bCKFull + s), 1);
-            mbar_init(bar(bCVFull + s), 1);
             mbar_init(bar(bCKEmpty + s), 4);
+        }
+        for (int s = 0; s < Lay::kCodeStagesV; ++s) {
+            mbar_init(bar(bCVFull + s), 1);
             mbar_init(bar(bCVEmpty + s), 4);
         }
         mbar_init(bar(bODone), 1);
@@ -314,16 +322,17 @@ __global__ void __launch_bounds__(TcLayout<Fp8>::kThreads, 1)
         // ------------------------------------------------------------ producer
         if (f16ops && lane < 2 && n_tiles > 0) {
             // E4M3 items: lane 0 loads the K codes, lane 1 the V codes, each into its
-            // own 2-stage staging ring (a stage is free once the converters read it).
+            // own staging ring (a stage is free once the converters have read it).
             const bool is_k = lane == 0;
+            const int ns = is_k ? Lay::kCodeStagesK : Lay::kCodeStagesV;
             const int cfull = is_k ? bCKFull : bCVFull;
             const int cempty = is_k ? bCKEmpty : bCVEmpty;
             const uint32_t ring = base + (is_k ? Lay::kOffCK : Lay::kOffCV);
             const CUtensorMap* m = is_k ? mk : mv;
             int issued = 0;
             for (int j = 0; j < n_tiles; ++j) {
-                const int cs = j & 1;
-                if (j >= 2 && !mbar_wait(bar(cempty + cs), ((j >> 1) - 1) & 1, abort_flag)) {
+                const int cs = j % ns;
+                if (j >= ns && !mbar_wait(bar(cempty + cs), ((j / ns) - 1) & 1, abort_flag)) {
                     tc_abort(p.err, abort_flag);
                     break;
                 }
@@ -332,8 +341,8 @@ __global__ void __launch_bounds__(TcLayout<Fp8>::kThreads, 1)
                 issued = j + 1;
             }
             // Let every load this thread issued land before the CTA can exit.
-            for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-                mbar_wait(bar(cfull + (j & 1)), (j >> 1) & 1, nullptr);
+            for (int j = (issued > ns ? issued - ns : 0); j < issued; ++j)
+                mbar_wait(bar(cfull + j % ns), (j / ns) & 1, nullptr);
         } else if (!f16ops && lane == 0 && n_tiles > 0) {
             // bf16 tiles straight into the operand rings.
             int issued = 0;
@@ -373,16 +382,17 @@ __global__ void __launch_bounds__(TcLayout<Fp8>::kThreads, 1)
         if (f16ops && n_tiles > 0) {
             const int cw = (warp - 6) & 3;
             const int kv = warp >= 10 ? 1 : 0;
+            const int ncs = kv ? Lay::kCodeStagesV : Lay::kCodeStagesK;
             bool ok = true;
             for (int j = 0; ok && j < n_tiles; ++j) {
-                const int cs = j & 1;  // staging stage
-                const int os = j & 1;  // operand stage (2 stages for E4M3 caches)
+                const int cs = j % ncs;  // staging stage
+                const int os = j & 1;    // operand stage (2 stages for E4M3 caches)
                 {
                     const int cfull = kv ? bCVFull : bCKFull;
                     const int cempty = kv ? bCVEmpty : bCKEmpty;
                     const int ofull = kv ? bVFull : bKFull;
                     const int oempty = kv ? bVEmpty : bKEmpty;
-                    if (!__all_sync(0xffffffffu, mbar_wait(bar(cfull + cs), (j >> 1) & 1, abort_flag)) ||
+                    if (!__all_sync(0xffffffffu, mbar_wait(bar(cfull + cs), (j / ncs) & 1, abort_flag)) ||
                         (j >= 2 &&
                          !__all_sync(0xffffffffu, mbar_wait(bar(oempty + os), ((j >> 1) - 1) & 1, abort_flag)))) {
                         if (lane == 0) tc_abort(p.err, abort_flag);
@@ -391,7 +401,7 @@ __global__ void __launch_bounds__(TcLayout<Fp8>::kThreads, 1)
                     }
                     const uint8_t* src = sb + (kv ? Lay::kOffCV : Lay::kOffCK) + cs * kTcCodeTile;
                     uint8_t* dst = sb + (kv ? Lay::kOffV : Lay::kOffK) + os * kTcTile;
-#pragma unroll 2
+#pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const int u = lane + 32 * i;
                         const int r = 32 * cw + (u >> 3);
