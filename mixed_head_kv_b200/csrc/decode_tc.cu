@@ -376,9 +376,9 @@ __global__ void __launch_bounds__(TcLayout<Fp8>::kThreads, 1)
     } else if (Fp8 && warp >= 6) {
         // ------------------------------------------------------------ converters (E4M3 items)
         // Warps 6-9 convert the K tiles, warps 10-13 the V tiles; warp c of a group
-        // converts rows [32c, 32c+32): 16 codes per lane and step (lanes 8r'..8r'+7
-        // cover one 128-byte row), written as 16 f16 into the row's two 16-byte
-        // chunks of the 128-byte-swizzled operand tile.
+        // converts rows [32c, 32c+32): 16 codes per lane and step (four rows per
+        // step), written as 16 f16 into the row's two 16-byte chunks of the
+        // 128-byte-swizzled operand tile.
         if (f16ops && n_tiles > 0) {
             const int cw = (warp - 6) & 3;
             const int kv = warp >= 10 ? 1 : 0;
@@ -401,11 +401,17 @@ __global__ void __launch_bounds__(TcLayout<Fp8>::kThreads, 1)
                     }
                     const uint8_t* src = sb + (kv ? Lay::kOffCV : Lay::kOffCK) + cs * kTcCodeTile;
                     uint8_t* dst = sb + (kv ? Lay::kOffV : Lay::kOffK) + os * kTcTile;
+                    // Lane -> (row, 16-code group): each quarter-warp takes two adjacent rows,
+                    // groups 0-3 of one and 4-7 of the other, so that its eight 16-byte code
+                    // loads and its eight swizzled f16 stores each land on eight distinct
+                    // 16-byte bank groups (one shared-memory wavefront per quarter).
+                    const int qw = lane >> 3;
+                    const int hr = (lane >> 2) & 1;
+                    const int row_l = 2 * (qw & 1) + hr;
+                    const int c16 = (lane & 3) + 4 * (hr ^ (qw >> 1));
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const int u = lane + 32 * i;
-                        const int r = 32 * cw + (u >> 3);
-                        const int c16 = u & 7;  // 16-code group of the row
+                        const int r = 32 * cw + 4 * i + row_l;
                         const uint4 c = *reinterpret_cast<const uint4*>(src + r * 128 + c16 * 16);
                         const uint4 lo = make_uint4(f16x2_from_e4m3x2(c.x & 0xFFFFu), f16x2_from_e4m3x2(c.x >> 16),
                                                     f16x2_from_e4m3x2(c.y & 0xFFFFu), f16x2_from_e4m3x2(c.y >> 16));
