@@ -133,7 +133,8 @@ typedef struct duo_cache duo_cache;
  *                         (num_q_heads / num_kv_heads) x (head_dim + 1) fp32,
  *                         R = the most retrieval KV heads of any one layer
  *                         (streaming heads write none); per-(sequence, KV head)
- *                         split counters; an error word
+ *                         split counters; an error word and the prefill's
+ *                         work-item counters (one 256-byte block)
  *   E4M3 scales           DUO_KV_E4M3 only: [num_layers][num_kv_heads] x 4 fp32
  *                         (k_scale, v_scale and their fp32 reciprocals), 1 until
  *                         duo_cache_set_kv_scales

@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libduo.so")
-SOURCES = ["duo_abi.cu", "append.cu", "decode.cu", "decode_tc.cu", "prefill.cu", "decode_static.cu"]
+SOURCES = ["duo_abi.cu", "append.cu", "decode.cu", "decode_tc.cu", "prefill.cu", "prefill_stream.cu", "decode_static.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

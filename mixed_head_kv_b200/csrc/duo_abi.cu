@@ -39,7 +39,7 @@ Regions regions_for(const duo_layout& L, int64_t n_retr_all, int64_t n_strm_all,
     r.part_o = align_up(items * G * D * sizeof(float));
     r.part_lse = align_up(items * G * sizeof(float));
     r.counters = align_up(static_cast<size_t>(L.batch) * L.num_kv_heads * sizeof(uint32_t));
-    r.err = align_up(sizeof(uint32_t));
+    r.err = align_up(3 * sizeof(uint32_t));  // error word, prefill work counter and done counter
     // E4M3 caches: k_scale, v_scale and their reciprocals per (layer, KV head)
     r.scales = L.kv_format == DUO_KV_E4M3
                    ? align_up(static_cast<size_t>(L.num_layers) * L.num_kv_heads * 4 * sizeof(float))
@@ -502,6 +502,7 @@ duo_status prefill_impl(duo_cache* c, int32_t layer, const void* q, const void* 
     PrefillParams p{};
     p.out = static_cast<bf16*>(out);
     p.err = c->err;
+    p.work = c->err + 1;  // the error word's 256-byte region: words 1 and 2
     p.len = len0;
     p.C = static_cast<int32_t>(n_rows);
     p.ragged = uniform ? 0 : 1;

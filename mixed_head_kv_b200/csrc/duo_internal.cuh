@@ -183,6 +183,10 @@ constexpr int kTileK = 128;   // keys per KV tile
 struct PrefillParams {
     bf16* out;  // [B][C][Hq][D]
     uint32_t* err;
+    // Two words, zero between launches: [0] next work item, [1] CTAs done (the
+    // last CTA of a launch zeroes both). The CTAs of one launch take items in
+    // order from [0], so launches on one cache must be stream-ordered.
+    uint32_t* work;
     int64_t len;  // tokens cached before the chunk (uniform batch)
     int32_t C;    // chunk length; rows per sequence of q, k, v and out
     int32_t B, Hq, Hkv, G, D, S, R, W;
@@ -208,6 +212,10 @@ struct PrefillMaps {
     CUtensorMap sv;
 };
 cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, int num_sms, cudaStream_t s);
+// The streaming-head work items of a prefill launch (prefill_stream.cu); `after_retrieval`:
+// launched behind the retrieval-item kernel with programmatic dependent launch.
+cudaError_t launch_prefill_streaming(const PrefillParams& p, const PrefillMaps& maps, int num_sms,
+                                     bool after_retrieval, cudaStream_t s);
 
 }  // namespace duo
 

@@ -47,7 +47,8 @@ DUO_MASK_FN RingVis ring_visible(int64_t len, int64_t sink, int64_t recent, int 
     if (lo < sink) lo = sink;
     const int64_t c = len - lo;
     if (c > 0) {
-        const int64_t r0 = (lo - sink) % recent;
+        // 0 <= lo - sink < len + qrow < 2^31 and recent < 2^31: a 32-bit remainder.
+        const int64_t r0 = static_cast<int64_t>(static_cast<uint32_t>(lo - sink) % static_cast<uint32_t>(recent));
         g.a0 = sink + r0;
         if (r0 + c <= recent) {
             g.b0 = sink + r0 + c;

@@ -1,8 +1,13 @@
 // prefill.cu — mixed-head attention of one prefill chunk (DuoAttention
-// pre-filling), retrieval and streaming heads in one launch, on tcgen05.
+// pre-filling) on tcgen05: the retrieval heads' work items, one per CTA, and
+// the launch of both prefill kernels.
 //
-// One CTA = one (batch, query head, 128-query tile) work item. Retrieval items
-// come first, heaviest (last query tile) first; streaming items fill in behind.
+// Work item = one (batch, query head, 128-query tile). This kernel runs the
+// retrieval items, one per CTA, heaviest (last query tile) first; the streaming
+// items (a few key tiles each, so a CTA start, a Q load and an epilogue per item
+// would weigh on them) run in prefill_stream.cu's persistent kernel, launched
+// right behind this one with programmatic dependent launch: its CTAs take the
+// SMs that this grid's CTAs leave.
 //
 // Key tiles of 128 keys are listed per item and fully masked tiles are never
 // listed:
@@ -39,19 +44,12 @@
 // All operand tiles in shared memory are 128-byte swizzled (TMA writes them,
 // the MMA reads them through descriptors). Every mbarrier wait is time-bounded;
 // on timeout the CTA records kErrPrefillWait and unwinds.
-#include "duo_internal.cuh"
-#include "mask_rules.cuh"
-#include "sm100.cuh"
-#include "tile_plan.cuh"
+#include "prefill_common.cuh"
 
 namespace duo {
 
 namespace {
 
-constexpr int kThreads = 384;
-constexpr int kTileBytesPerColBlock = kTileQ * 128;  // 128 rows x 64 bf16 (128 B)
-constexpr float kRescaleThreshold = 8.0f;             // log2 units: rescale when max grows by > 2^8
-constexpr int kHalf = kTileK / 2;                     // keys per softmax thread and tile
 
 template <int D>
 struct Layout {
@@ -86,42 +84,6 @@ constexpr int kDrain = 17;
 // needs S(j+2), which needs both PV halves of tile j to have consumed P(j)) and
 // the output waits on a single-phase barrier.
 
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemO = 256;  // O of key half h at kTmemO + h * D
-constexpr uint32_t kTmemP = 32;   // P of a key tile at its S buffer + 32 (64 columns of bf16 pairs)
-
-__device__ __forceinline__ void record_abort(uint32_t* err, volatile int* abort_flag) {
-    *abort_flag = 1;
-    atomicOr(err, kErrPrefillWait);
-}
-
-// Visibility of keys [32w, 32w+32) of tile (src, row0) from chunk query row
-// `qrow`: src 0 retrieval cache, 1 streaming cache, 2 chunk (mask_rules.cuh).
-__device__ __forceinline__ uint32_t visible_bits(const PrefillParams& p, const Item& it, int src, int row0, int w,
-                                                 int qrow, const RingVis& ring) {
-    const int64_t base = row0 + 32 * w;
-    if (src == 0) return retrieval_cache_bits(it.L, base);
-    if (src == 2) return chunk_bits(it.retr, it.L, it.C, p.S, p.R, qrow, base);
-    return streaming_cache_bits(it.L, p.S, ring, base);
-}
-
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
-// D[tmem] (+)= A[tmem] * B[smem], kind::f16: the PV product with P held in TMEM.
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // Named barrier over the two warps (64 threads) that share one row quarter.
 __device__ __forceinline__ void pair_sync(int quarter) {
     asm volatile("bar.sync %0, 64;" ::"r"(1 + quarter) : "memory");
@@ -143,6 +105,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sbase + Lay::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + Lay::kMisc + 4);
 
+    // The streaming-item kernel behind this one reads nothing this grid writes: it
+    // may start as soon as every CTA of this grid is resident.
+    grid_launch_dependents();
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
@@ -458,25 +423,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D>
-cudaError_t launch_d(const PrefillParams& p, const PrefillMaps& maps, cudaStream_t s) {
+cudaError_t launch_d(const PrefillParams& p, const PrefillMaps& maps, int n_items, cudaStream_t s) {
     // Same shared-memory request for every D: one CTA per SM, so a CTA never
     // waits on another for TMEM columns.
     const int smem = Layout<128>::kAlloc;
     static SmemLimitOnce limit;
     cudaError_t e = limit.apply(reinterpret_cast<const void*>(&prefill_kernel<D>), smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = static_cast<unsigned>(p.B * p.Hq * p.n_qt);
-    prefill_kernel<D><<<grid, kThreads, smem, s>>>(p, maps);
+    prefill_kernel<D><<<static_cast<unsigned>(n_items), kThreads, smem, s>>>(p, maps);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, int /*num_sms*/, cudaStream_t s) {
-    if (p.B * p.Hq * p.n_qt == 0) return cudaSuccess;
-    if (p.D == 128) return launch_d<128>(p, maps, s);
-    if (p.D == 64) return launch_d<64>(p, maps, s);
-    return cudaErrorInvalidValue;
+cudaError_t launch_prefill(const PrefillParams& p, const PrefillMaps& maps, int num_sms, cudaStream_t s) {
+    if (p.D != 128 && p.D != 64) return cudaErrorInvalidValue;
+    const int n_retr_items = p.B * p.n_retr_q * p.n_qt;
+    const int n_strm_items = p.B * (p.Hq - p.n_retr_q) * p.n_qt;
+    if (n_retr_items > 0) {
+        const cudaError_t e = p.D == 128 ? launch_d<128>(p, maps, n_retr_items, s) : launch_d<64>(p, maps, n_retr_items, s);
+        if (e != cudaSuccess) return e;
+    }
+    if (n_strm_items > 0) return launch_prefill_streaming(p, maps, num_sms, n_retr_items > 0, s);
+    return cudaSuccess;
 }
 
 }  // namespace duo
