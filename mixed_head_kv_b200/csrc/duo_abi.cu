@@ -538,6 +538,7 @@ duo_status prefill_impl(duo_cache* c, int32_t layer, const void* q, const void* 
     maps.sk = c->map_sk;
     maps.sv = c->map_sv;
     if (!make_chunk_map(&maps.q, q, L.head_dim, L.num_q_heads, n_rows, L.batch) ||
+        !make_chunk_map(&maps.out, out, L.head_dim, L.num_q_heads, n_rows, L.batch) ||
         !make_chunk_map(&maps.k, k, L.head_dim, L.num_kv_heads, n_rows, L.batch) ||
         !make_chunk_map(&maps.v, v, L.head_dim, L.num_kv_heads, n_rows, L.batch))
         return DUO_ERR_CUDA;

@@ -204,6 +204,7 @@ struct PrefillParams {
 
 struct PrefillMaps {
     CUtensorMap q;   // chunk q  (D, Hq, C, B), box (64, 1, 128, 1)
+    CUtensorMap out; // prefill output, same shape and box as q (tile stores)
     CUtensorMap k;   // chunk k  (D, Hkv, C, B)
     CUtensorMap v;
     CUtensorMap rk;  // retrieval pool (D, max_len, n_retr_all*B), box (64, 128, 1)

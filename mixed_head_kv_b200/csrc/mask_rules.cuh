@@ -85,4 +85,50 @@ DUO_MASK_FN uint32_t chunk_bits(int retr, int64_t len, int64_t C, int64_t sink, 
     return causal & (sinks | band);
 }
 
+// The same rules with every bound of one query row computed once, in 32-bit
+// arithmetic, for kernels that test many words of a row: chunk rows and slot
+// indices are below 2^30 (chunk and window sizes), cache positions below 2^31.
+// Each *_row function returns exactly what its 64-bit counterpart above returns
+// for the same row and word.
+DUO_MASK_FN uint32_t bits_below32(int32_t x) {
+    if (x <= 0) return 0u;
+    if (x >= 32) return 0xFFFFFFFFu;
+    return (1u << static_cast<uint32_t>(x)) - 1u;
+}
+
+struct RowVis {
+    int32_t c_hi;            // chunk rows < c_hi are causal: min(qrow, C - 1) + 1
+    int32_t c_sink;          // chunk rows < c_sink hold sinks (streaming): max(sink - len, 0)
+    int32_t c_lo;            // chunk rows >= c_lo are inside the window: qrow - recent + 1 (retrieval: -2^30)
+    int32_t s_sink;          // streaming cache: sink slots < min(len, sink) are valid
+    int32_t a0, b0, a1, b1;  // streaming cache: visible ring slot ranges (ring_visible)
+    int32_t r_len;           // retrieval cache: slots < len are valid
+};
+
+DUO_MASK_FN RowVis row_visible(int retr, int64_t len, int64_t C, int64_t sink, int64_t recent, int qrow) {
+    RowVis v;
+    v.c_hi = static_cast<int32_t>((qrow < C - 1 ? qrow : C - 1) + 1);
+    v.c_sink = retr ? 0 : static_cast<int32_t>(len < sink ? sink - len : 0);
+    v.c_lo = retr ? -(1 << 30) : static_cast<int32_t>(qrow - recent + 1);
+    v.s_sink = static_cast<int32_t>(len < sink ? len : sink);
+    const RingVis g = ring_visible(len, sink, recent, qrow);
+    v.a0 = static_cast<int32_t>(g.a0);
+    v.b0 = static_cast<int32_t>(g.b0);
+    v.a1 = static_cast<int32_t>(g.a1);
+    v.b1 = static_cast<int32_t>(g.b1);
+    v.r_len = static_cast<int32_t>(len);
+    return v;
+}
+
+DUO_MASK_FN uint32_t retrieval_cache_bits_row(const RowVis& v, int32_t base) { return bits_below32(v.r_len - base); }
+
+DUO_MASK_FN uint32_t streaming_cache_bits_row(const RowVis& v, int32_t base) {
+    return bits_below32(v.s_sink - base) | (bits_below32(v.b0 - base) & ~bits_below32(v.a0 - base)) |
+           (bits_below32(v.b1 - base) & ~bits_below32(v.a1 - base));
+}
+
+DUO_MASK_FN uint32_t chunk_bits_row(const RowVis& v, int32_t base) {
+    return bits_below32(v.c_hi - base) & (bits_below32(v.c_sink - base) | ~bits_below32(v.c_lo - base));
+}
+
 }  // namespace duo

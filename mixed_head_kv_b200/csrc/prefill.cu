@@ -58,7 +58,8 @@ struct Layout {
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kTile;       // 2 stages
     static constexpr int kV = kK + 2 * kTile;   // 2 stages
-    static constexpr int kBar = kV + 2 * kTile;
+    static constexpr int kO = kV + 2 * kTile;   // output tile staged for the tile store
+    static constexpr int kBar = kO + kTile;
     // Pair exchange: maxima [tile parity][half][row], ok flags [parity][half][quarter],
     // row sums [half][row].
     static constexpr int kXchg = kBar + 32 * 8;
@@ -66,6 +67,7 @@ struct Layout {
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
+static_assert(Layout<128>::kAlloc <= 227 * 1024, "shared memory of one CTA");
 
 // mbarrier indices
 constexpr int kQFull = 0;
@@ -79,6 +81,7 @@ constexpr int kP1Full = 13;    // + S buffer: P of keys 64-127 written (4 arriva
 constexpr int kODone = 15;     // one phase per key tile (both PV halves)
 constexpr int kOFinal = 16;    // one phase, after the last PV
 constexpr int kDrain = 17;
+constexpr int kStaged = 18;    // the output tile is staged (8 arrivals: softmax warps)
 // Every barrier is waited with a phase parity, so none may complete two phases
 // beyond the one its waiter waits for: S and P barriers are per S buffer (P(j+2)
 // needs S(j+2), which needs both PV halves of tile j to have consumed P(j)) and
@@ -128,6 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar(kODone), 1);
         mbar_init(bar(kOFinal), 1);
         mbar_init(bar(kDrain), 1);
+        mbar_init(bar(kStaged), 8);
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -256,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int qrow = it.q0 + row;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t tO = tmem + lane_base + kTmemO + h * D;
-        const RingVis ring = ring_visible(it.L, p.S, p.R, qrow);
+        const RowVis vis = row_visible(it.retr, it.L, it.C, p.S, p.R, qrow);
         const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
         volatile float* xm = xchg;        // [half][row] running max
         volatile float* xl = xchg + 256;  // [half][row] row sum
@@ -295,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!full) {
 #pragma unroll
                 for (int w = 0; w < 2; ++w) {
-                    const uint32_t bits = visible_bits(p, it, src, row0, 2 * h + w, qrow, ring);
+                    const uint32_t bits = visible_bits(vis, src, row0 + 32 * (2 * h + w));
                     live[w] = __any_sync(0xffffffffu, bits != 0u);
                     if (live[w] && !__all_sync(0xffffffffu, bits == 0xFFFFFFFFu)) {
 #pragma unroll
@@ -389,6 +393,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float f1 = (h == 0 ? f_o : f_self) * inv;
         if (__all_sync(0xffffffffu, ok && mbar_wait(bar(kOFinal), 0, abort_flag))) {
             tc_fence_after();
+            // A tile whose 128 rows are all output rows goes out as one tile store from
+            // shared memory (128-byte swizzled), issued by one thread once every
+            // softmax warp has staged its part; other tiles (the last rows of a
+            // sequence's chunk) are stored row by row.
+            const bool tile_store = it.q0 + kTileQ <= it.C;
             const uint32_t tO0 = tmem + lane_base + kTmemO + h * (D / 2);
             bf16* orow = p.out + ((static_cast<int64_t>(it.b) * p.C + qrow) * p.Hq + it.head) * D + h * (D / 2);
             uint32_t r0[32], r1[32];
@@ -397,18 +406,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(tO0 + c * 32, r0);
                 tmem_ld32(tO0 + D + c * 32, r1);
                 tc_wait_ld();
-                if (qrow < it.C) {
 #pragma unroll
-                    for (int v8 = 0; v8 < 4; ++v8) {
-                        uint32_t w[4];
+                for (int v8 = 0; v8 < 4; ++v8) {
+                    uint32_t w[4];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int e = v8 * 8 + 2 * i;
-                            w[i] = pack_bf16x2(__uint_as_float(r0[e]) * f0 + __uint_as_float(r1[e]) * f1,
-                                               __uint_as_float(r0[e + 1]) * f0 + __uint_as_float(r1[e + 1]) * f1);
-                        }
+                    for (int i = 0; i < 4; ++i) {
+                        const int e = v8 * 8 + 2 * i;
+                        w[i] = pack_bf16x2(__uint_as_float(r0[e]) * f0 + __uint_as_float(r1[e]) * f1,
+                                           __uint_as_float(r0[e + 1]) * f0 + __uint_as_float(r1[e + 1]) * f1);
+                    }
+                    if (tile_store) {
+                        const int col = h * (D / 2) + c * 32 + v8 * 8;
+                        const int off = (col >> 6) * kTileBytesPerColBlock + row * 128 +
+                                        ((((col & 63) >> 3) ^ (row & 7)) << 4);
+                        *reinterpret_cast<uint4*>(sbase + Lay::kO + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                    } else if (qrow < it.C) {
                         *reinterpret_cast<uint4*>(orow + c * 32 + v8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
+                }
+            }
+            if (tile_store) fence_proxy_async_smem();  // generic writes -> visible to the tile store
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kStaged));
+            if (warp == 0 && lane == 0) {
+                if (mbar_wait(bar(kStaged), 0, abort_flag)) {
+                    if (tile_store) {
+                        for (int kb = 0; kb < Lay::kColBlocks; ++kb)
+                            tma_store_4d(&maps.out, base + Lay::kO + kb * kTileBytesPerColBlock, kb * 64, it.head,
+                                         it.q0, it.b);
+                        bulk_commit_group();
+                        bulk_wait_group0();  // completes before the CTA exits
+                    }
+                } else {
+                    record_abort(p.err, abort_flag);
                 }
             }
         } else {

@@ -28,14 +28,13 @@ __device__ __forceinline__ void record_abort(uint32_t* err, volatile int* abort_
     atomicOr(err, kErrPrefillWait);
 }
 
-// Visibility of keys [32w, 32w+32) of tile (src, row0) from chunk query row
-// `qrow`: src 0 retrieval cache, 1 streaming cache, 2 chunk (mask_rules.cuh).
-__device__ __forceinline__ uint32_t visible_bits(const PrefillParams& p, const Item& it, int src, int row0, int w,
-                                                 int qrow, const RingVis& ring) {
-    const int64_t base = row0 + 32 * w;
-    if (src == 0) return retrieval_cache_bits(it.L, base);
-    if (src == 2) return chunk_bits(it.retr, it.L, it.C, p.S, p.R, qrow, base);
-    return streaming_cache_bits(it.L, p.S, ring, base);
+// Visibility of the 32 keys from `base` of a tile from `src` (0 retrieval
+// cache, 1 streaming cache, 2 chunk) for one query row, from its row bounds
+// (mask_rules.cuh).
+__device__ __forceinline__ uint32_t visible_bits(const RowVis& v, int src, int32_t base) {
+    if (src == 2) return chunk_bits_row(v, base);
+    if (src == 1) return streaming_cache_bits_row(v, base);
+    return retrieval_cache_bits_row(v, base);
 }
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

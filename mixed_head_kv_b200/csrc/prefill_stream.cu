@@ -67,7 +67,8 @@ struct Layout {
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kTile;              // kKStages stages
     static constexpr int kV = kK + kKStages * kTile;   // 2 stages
-    static constexpr int kBar = kV + 2 * kTile;
+    static constexpr int kO = kV + 2 * kTile;    // output tile staged for the tile store
+    static constexpr int kBar = kO + kTile;
     // Epilogue exchange of the two halves of a row: maxima and row sums
     // [item parity][half][row].
     static constexpr int kXchg = kBar + 40 * 8;
@@ -77,6 +78,7 @@ struct Layout {
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
+static_assert(Layout<128>::kAlloc <= 227 * 1024, "shared memory of one CTA");
 
 // mbarrier indices
 constexpr int kQFull = 0;       // one phase per item
@@ -95,6 +97,8 @@ constexpr int kDrain = 21;
 constexpr int kItemFull = 22;   // + queue slot: work item published (producer)
 constexpr int kItemEmpty = 26;  // + queue slot: read by every consumer (kConsumers arrivals)
 constexpr int kPair = 30;       // + row quarter: both halves of the rows wrote their max and sum (2 arrivals)
+constexpr int kStaged = 34;     // one phase per item: the output tile is staged (8 arrivals: softmax warps)
+constexpr int kOFree = 35;      // one phase per item: the previous item's tile store has read the staging tile
 constexpr int kQueueSlots = 4;
 constexpr int kConsumers = 10;  // V producer, MMA issuer, 8 softmax warps
 // Every barrier is waited with a phase parity, so none may complete two phases
@@ -151,6 +155,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar(kItemEmpty + s), kConsumers);
             mbar_init(bar(kPair + s), 2);  // s = row quarter
         }
+        mbar_init(bar(kStaged), 8);
+        mbar_init(bar(kOFree), 1);
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
@@ -416,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Item it = make_item(p, idx);
             const int n = it.n_tiles;
             const int qrow = it.q0 + row;
-            const RingVis ring = ring_visible(it.L, p.S, p.R, qrow);
+            const RowVis vis = row_visible(it.retr, it.L, it.C, p.S, p.R, qrow);
             float m_run = -INFINITY;
             float l_run = 0.f;
             for (int j = 0; j < n; ++j, ++g) {
@@ -451,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!full) {
 #pragma unroll
                     for (int w = 0; w < 2; ++w) {
-                        const uint32_t bits = visible_bits(p, it, src, row0, 2 * h + w, qrow, ring);
+                        const uint32_t bits = visible_bits(vis, src, row0 + 32 * (2 * h + w));
                         live[w] = __any_sync(0xffffffffu, bits != 0u);
                         if (live[w] && !__all_sync(0xffffffffu, bits == 0xFFFFFFFFu)) {
 #pragma unroll
@@ -563,6 +569,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            // A tile whose 128 rows are all output rows goes out as one tile store from
+            // shared memory (128-byte swizzled like the operand tiles); other tiles
+            // (the last rows of a sequence's chunk) are stored row by row. One
+            // thread issues the stores; the staging tile is rewritten only after the
+            // previous item's store has read it, and the phases of kOFree (arrived
+            // after the issuer's own wait on this item's O) never run ahead of a
+            // warp that has yet to wait on them.
+            const bool issuer = warp == 0 && lane == 0;
+            if (issuer) {
+                bulk_wait_group_read0();
+                mbar_arrive(bar(kOFree));
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(kOFree), ord & 1, abort_flag))) {
+                ok = false;
+                record_abort(p.err, abort_flag);
+                break;
+            }
+            const bool tile_store = it.q0 + kTileQ <= it.C;
             const uint32_t tO0 = tmem + lane_base + kTmemO + h * (D / 2);
             bf16* orow = p.out + ((static_cast<int64_t>(it.b) * p.C + qrow) * p.Hq + it.head) * D + h * (D / 2);
             uint32_t r0[32], r1[32];
@@ -571,18 +595,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(tO0 + c * 32, r0);
                 tmem_ld32(tO0 + D + c * 32, r1);
                 tc_wait_ld();
-                if (qrow < it.C) {
 #pragma unroll
-                    for (int v8 = 0; v8 < 4; ++v8) {
-                        uint32_t w[4];
+                for (int v8 = 0; v8 < 4; ++v8) {
+                    uint32_t w[4];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int e = v8 * 8 + 2 * i;
-                            w[i] = pack_bf16x2(__uint_as_float(r0[e]) * f0 + __uint_as_float(r1[e]) * f1,
-                                               __uint_as_float(r0[e + 1]) * f0 + __uint_as_float(r1[e + 1]) * f1);
-                        }
+                    for (int i = 0; i < 4; ++i) {
+                        const int e = v8 * 8 + 2 * i;
+                        w[i] = pack_bf16x2(__uint_as_float(r0[e]) * f0 + __uint_as_float(r1[e]) * f1,
+                                           __uint_as_float(r0[e + 1]) * f0 + __uint_as_float(r1[e + 1]) * f1);
+                    }
+                    if (tile_store) {
+                        const int col = h * (D / 2) + c * 32 + v8 * 8;
+                        const int off = (col >> 6) * kTileBytesPerColBlock + row * 128 +
+                                        ((((col & 63) >> 3) ^ (row & 7)) << 4);
+                        *reinterpret_cast<uint4*>(sbase + Lay::kO + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                    } else if (qrow < it.C) {
                         *reinterpret_cast<uint4*>(orow + c * 32 + v8 * 8) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
+                }
+            }
+            if (tile_store) fence_proxy_async_smem();  // generic writes -> visible to the tile store
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kStaged));
+            if (issuer) {
+                if (mbar_wait(bar(kStaged), ord & 1, abort_flag)) {
+                    if (tile_store) {
+                        for (int kb = 0; kb < Lay::kColBlocks; ++kb)
+                            tma_store_4d(&maps.out, base + Lay::kO + kb * kTileBytesPerColBlock, kb * 64, it.head,
+                                         it.q0, it.b);
+                        bulk_commit_group();
+                    }
+                } else {
+                    ok = false;
+                    record_abort(p.err, abort_flag);
                 }
             }
             // O is read: the next item's first PV may overwrite it.
@@ -590,6 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kOEmpty));
         }
+        if (warp == 0 && lane == 0) bulk_wait_group0();  // every tile store completes before the CTA exits
     }
 
     tc_fence_before();
