@@ -72,9 +72,11 @@ struct Layout {
     // Epilogue exchange of the two halves of a row: maxima and row sums
     // [item parity][half][row].
     static constexpr int kXchg = kBar + 40 * 8;
-    // Work items handed to the roles [slot], then the MMA issuer's tile counts [slot].
+    // Work items handed to the roles: item index [slot], the MMA issuer's tile
+    // counts [slot], then the items themselves [slot].
     static constexpr int kQueue = kXchg + 2 * 2 * 2 * 128 * 4;
-    static constexpr int kMisc = kQueue + 16 * 4;
+    static constexpr int kItems = kQueue + 16 * 4;
+    static constexpr int kMisc = kItems + 4 * static_cast<int>(sizeof(Item));
     static constexpr int kBytes = kMisc + 64;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
@@ -123,6 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto bar = [&](int i) { return base + Lay::kBar + 8u * i; };
     volatile float* xchg = reinterpret_cast<volatile float*>(sbase + Lay::kXchg);
     volatile int* queue = reinterpret_cast<volatile int*>(sbase + Lay::kQueue);
+    Item* items = reinterpret_cast<Item*>(sbase + Lay::kItems);  // written before, read after the slot's barrier
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sbase + Lay::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + Lay::kMisc + 4);
 
@@ -170,13 +173,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // Item `ord` of this CTA from the queue (-1: no more work, or the wait gave up).
-    // Every consumer reads each slot once and then frees it.
-    auto take_item = [&](int ord, bool arrive) -> int {
+    // Item `ord` of this CTA from the queue: its index (-1: no more work, -2: the
+    // wait gave up) and, for an index >= 0, the item itself. Every consumer reads
+    // each slot once and then frees it.
+    auto take_item = [&](int ord, Item& out) -> int {
         const int slot = ord % kQueueSlots;
         if (!mbar_wait(bar(kItemFull + slot), (ord / kQueueSlots) & 1, abort_flag)) return -2;
         const int idx = queue[slot];
-        if (arrive) mbar_arrive(bar(kItemEmpty + slot));
+        if (idx >= 0) out = items[slot];
+        mbar_arrive(bar(kItemEmpty + slot));
         return idx;
     };
 
@@ -209,7 +214,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 queue[slot] = idx;
-                mbar_arrive(bar(kItemFull + slot));  // release: the consumers see queue[slot]
+                if (idx >= 0) items[slot] = it;
+                mbar_arrive(bar(kItemFull + slot));  // release: the consumers see queue[slot] and items[slot]
                 if (idx < 0) break;
                 // Q of the previous item is free once its last QK has run (the MMA
                 // issuer starts this item's QKs only after that item's last PV).
@@ -255,10 +261,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int g = 0, issued = 0;
             for (int ord = 0;; ++ord) {
-                const int idx = take_item(ord, true);
+                Item it;
+                const int idx = take_item(ord, it);
                 if (idx == -2) record_abort(p.err, abort_flag);
                 if (idx < 0) break;
-                const Item it = make_item(p, idx);
                 bool ok = true;
                 for (int j = 0; j < it.n_tiles; ++j, ++g) {
                     const int st = g & 1;
@@ -306,14 +312,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (qk_end) return 0;
                 if (qk_j == qk_n) {
                     if (pv_g != qk_g) return 0;
-                    const int idx = take_item(qk_ord, true);
+                    Item it;
+                    const int idx = take_item(qk_ord, it);
                     if (idx == -2) return -1;
                     if (idx < 0) {
                         qk_end = true;
                         return 0;
                     }
                     qk_cur = qk_ord++;
-                    qk_n = make_item(p, idx).n_tiles;
+                    qk_n = it.n_tiles;
                     n_of[qk_cur % kQueueSlots] = qk_n;
                     qk_j = 0;
                     if (!mbar_wait(bar(kQFull), qk_cur & 1, abort_flag)) return -1;
@@ -410,19 +417,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t scale2 = f2pack(p.scale_log2, p.scale_log2);
         bool ok = true;
         int g = 0;  // key tiles of this CTA so far
-        for (int ord = 0; ok; ++ord) {
-            int idx = -1;
-            if (lane == 0) idx = take_item(ord, true);
-            idx = __shfl_sync(0xffffffffu, idx, 0);
-            if (idx == -2) {
-                ok = false;
-                record_abort(p.err, abort_flag);
-            }
-            if (idx < 0) break;
-            const Item it = make_item(p, idx);
+        // The warp's lanes read a queue slot together, then lane 0 frees it.
+        auto take = [&](int ord, Item& out) -> int {
+            const int slot = ord % kQueueSlots;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(kItemFull + slot), (ord / kQueueSlots) & 1, abort_flag)))
+                return -2;
+            const int idx = queue[slot];
+            if (idx >= 0) out = items[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kItemEmpty + slot));
+            return idx;
+        };
+        Item it{};
+        int idx = take(0, it);
+        RowVis vis = row_visible(it.retr, it.L, it.C, p.S, p.R, it.q0 + row);
+        if (idx == -2) record_abort(p.err, abort_flag);
+        for (int ord = 0; ok && idx >= 0; ++ord) {
             const int n = it.n_tiles;
             const int qrow = it.q0 + row;
-            const RowVis vis = row_visible(it.retr, it.L, it.C, p.S, p.R, qrow);
             float m_run = -INFINITY;
             float l_run = 0.f;
             for (int j = 0; j < n; ++j, ++g) {
@@ -540,6 +552,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 record_abort(p.err, abort_flag);
                 break;
             }
+            // The next item (taken and its row bounds computed while this item's last PV
+            // runs, before the epilogue waits for it).
+            Item nit{};
+            const int nidx = take(ord + 1, nit);
+            const RowVis nvis = row_visible(nit.retr, nit.L, nit.C, p.S, p.R, nit.q0 + row);
             // Combine the halves: O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)),
             // each thread of a pair writing D/2 of the row's columns. The exchange
             // buffers alternate between items, so a fast pair member never overwrites
@@ -634,6 +651,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kOEmpty));
+            if (nidx == -2) {
+                ok = false;
+                record_abort(p.err, abort_flag);
+            }
+            idx = nidx;
+            it = nit;
+            vis = nvis;
         }
         if (warp == 0 && lane == 0) bulk_wait_group0();  // every tile store completes before the CTA exits
     }
