@@ -24,6 +24,7 @@
 
 #include "duo_internal.cuh"
 #include "sm100.cuh"
+#include "decode_merge.cuh"
 
 namespace duo {
 
@@ -607,78 +608,8 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
     __syncthreads();
     if (!*sm_last) return;
     __threadfence();
-    // The partials of this (b, KV head) are contiguous: [nsplit][G][D] floats and
-    // [nsplit][G] log-sum-exps. First every split's weight per head, from one
-    // coalesced load of the log-sum-exps: w = 2^(lse - max) / sum over the splits
-    // (a split without rows, lse = -inf, weighs 0). Then each thread sums its
-    // float4 unit over a subset of the splits, its loads independent of each
-    // other, and the subsets are added.
-    const int64_t item0 = (static_cast<int64_t>(b) * p.n_retr + ri) * p.nsplit;
-    const int ns = p.nsplit;
-    constexpr int kUnits = G * D / 4;  // float4 units of one split's partial
-    constexpr int kRep = kUnits >= kDecodeThreads ? 1 : kDecodeThreads / kUnits;
-    float4* sm_acc = reinterpret_cast<float4*>(smem);                  // [kRep][kUnits]
-    float* sm_w = reinterpret_cast<float*>(sm_acc + kRep * kUnits);    // [ns][G] log-sum-exps, then weights
-    float* sm_norm = sm_w + kDecodeMaxSplits * G;                      // [G] max, [G] 1 / sum
-    const float4* po = reinterpret_cast<const float4*>(p.part_o + item0 * G * D);
-    const float* pl = p.part_lse + item0 * G;
     __syncthreads();  // the per-warp merge arrays above are no longer read
-    for (int i = tid; i < ns * G; i += kDecodeThreads) sm_w[i] = __ldcg(pl + i);
-    __syncthreads();
-    for (int h = warp; h < G; h += kWarps) {
-        float M = -INFINITY;
-        for (int sp = lane; sp < ns; sp += 32) M = fmaxf(M, sm_w[sp * G + h]);
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        float S = 0.f;
-        for (int sp = lane; sp < ns; sp += 32) {
-            const float x = sm_w[sp * G + h];
-            S += (x == -INFINITY) ? 0.f : fast_exp2(x - M);
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) S += __shfl_xor_sync(0xffffffffu, S, off);
-        if (lane == 0) {
-            sm_norm[h] = M;
-            sm_norm[G + h] = 1.f / S;  // S >= 1: the split holding the maximum weighs 1
-        }
-    }
-    __syncthreads();
-    for (int i = tid; i < ns * G; i += kDecodeThreads) {
-        const int h = i % G;
-        const float x = sm_w[i];
-        sm_w[i] = (x == -INFINITY) ? 0.f : fast_exp2(x - sm_norm[h]) * sm_norm[G + h];
-    }
-    __syncthreads();
-    for (int u = tid % kUnits; u < kUnits; u += kDecodeThreads) {
-        const int h = (u * 4) / D;
-        const int rep = tid / kUnits;  // < kRep
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int sp = rep; sp < ns; sp += kRep) {
-            const float w = sm_w[sp * G + h];
-            const float4 o = __ldcg(po + static_cast<int64_t>(sp) * kUnits + u);
-            acc.x = fmaf(w, o.x, acc.x);
-            acc.y = fmaf(w, o.y, acc.y);
-            acc.z = fmaf(w, o.z, acc.z);
-            acc.w = fmaf(w, o.w, acc.w);
-        }
-        sm_acc[rep * kUnits + u] = acc;
-    }
-    __syncthreads();
-    for (int u = tid; u < kUnits; u += kDecodeThreads) {
-        float4 acc = sm_acc[u];
-        for (int r = 1; r < kRep; ++r) {
-            const float4 x = sm_acc[r * kUnits + u];
-            acc.x += x.x;
-            acc.y += x.y;
-            acc.z += x.z;
-            acc.w += x.w;
-        }
-        const int h = (u * 4) / D;
-        const int d = (u * 4) % D;
-        bf16* o = p.out + (static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d;
-        *reinterpret_cast<uint2*>(o) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-    }
+    merge_split_partials<G, D, kDecodeThreads>(p, b, g, ri, smem);
     if (tid == 0) p.counters[b * p.Hkv + g] = 0u;  // ready for the next step (stream-ordered)
 }
 

@@ -45,6 +45,7 @@
 
 #include "duo_internal.cuh"
 #include "sm100.cuh"
+#include "decode_merge.cuh"
 
 namespace duo {
 
@@ -628,7 +629,7 @@ __global__ void __launch_bounds__(TcLayout<Fp8>::kThreads, 1)
     if (!is_retr || p.nsplit == 1) return;
 
     // Split-KV merge (D4): the last CTA of this (b, KV head) combines the
-    // partials, thread t column t of every head.
+    // partials (decode_merge.cuh), in the shared memory of the operand rings.
     __threadfence();
     __syncthreads();
     if (tid == 0) {
@@ -638,28 +639,7 @@ __global__ void __launch_bounds__(TcLayout<Fp8>::kThreads, 1)
     __syncthreads();
     if (!*last_flag) return;
     __threadfence();
-    if (tid < D) {
-        const int64_t item0 = (static_cast<int64_t>(b) * p.n_retr + ri) * p.nsplit;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            float M = -INFINITY, Ls = 0.f, acc = 0.f;
-#pragma unroll 4
-            for (int s = 0; s < p.nsplit; ++s) {
-                const float x = __ldcg(p.part_lse + (item0 + s) * G + h);
-                const float o = __ldcg(p.part_o + ((item0 + s) * G + h) * D + tid);
-                if (x > M) {
-                    const float f = fast_exp2(M - x);  // 0 while M is -inf
-                    Ls *= f;
-                    acc *= f;
-                    M = x;
-                }
-                const float w = (x == -INFINITY) ? 0.f : fast_exp2(x - M);
-                Ls += w;
-                acc = fmaf(w, o, acc);
-            }
-            p.out[(static_cast<int64_t>(b) * p.Hq + g * G + h) * D + tid] = __float2bfloat16_rn(acc / Ls);
-        }
-    }
+    merge_split_partials<G, kTcD, Lay::kThreads>(p, b, g, ri, sb);
     if (tid == 0) p.counters[b * p.Hkv + g] = 0u;  // ready for the next step (stream-ordered)
 }
 
