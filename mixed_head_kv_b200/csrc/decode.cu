@@ -598,17 +598,9 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p) {
     }
     if (final_now) return;
 
-    // Split-KV merge (D4): the last CTA of this (b, KV head) combines the partials.
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const uint32_t prev = atomicAdd(&p.counters[b * p.Hkv + g], 1u);
-        *sm_last = (prev == static_cast<uint32_t>(p.nsplit - 1));
-    }
-    __syncthreads();
-    if (!*sm_last) return;
-    __threadfence();
-    __syncthreads();  // the per-warp merge arrays above are no longer read
+    // Split-KV merge (D4): the last CTA of this (b, KV head) combines the partials
+    // (the handshake's barriers also end every read of the per-warp arrays above).
+    if (!split_arrive(&p.counters[b * p.Hkv + g], static_cast<uint32_t>(p.nsplit), sm_last)) return;
     merge_split_partials<G, D, kDecodeThreads>(p, b, g, ri, smem);
     if (tid == 0) p.counters[b * p.Hkv + g] = 0u;  // ready for the next step (stream-ordered)
 }

@@ -9,6 +9,23 @@
 
 namespace duo {
 
+// The split handshake, by every thread of a CTA that has stored its partial:
+// the stores precede (a barrier, then thread 0's GPU-scope acq_rel fence) the
+// increment of the (sequence, KV head) counter; the CTA whose increment
+// completes the count acquires the other CTAs' partials (the same fence after
+// the increment, then a barrier) and returns true: it merges.
+__device__ __forceinline__ bool split_arrive(uint32_t* counter, uint32_t nsplit, volatile int* flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");
+        const bool last = atomicAdd(counter, 1u) == nsplit - 1;
+        if (last) asm volatile("fence.acq_rel.gpu;" ::: "memory");
+        *flag = last ? 1 : 0;
+    }
+    __syncthreads();
+    return *flag != 0;
+}
+
 // Called by every thread of the merging CTA (kThreads of them) after a barrier;
 // `smem` holds kThreads float4 + 2 * kThreads floats of scratch at least.
 // The partials of this (b, KV head) are contiguous: [nsplit][G][D] floats and

@@ -630,15 +630,7 @@ __global__ void __launch_bounds__(TcLayout<Fp8>::kThreads, 1)
 
     // Split-KV merge (D4): the last CTA of this (b, KV head) combines the
     // partials (decode_merge.cuh), in the shared memory of the operand rings.
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const uint32_t prev = atomicAdd(&p.counters[b * p.Hkv + g], 1u);
-        *last_flag = (prev == static_cast<uint32_t>(p.nsplit - 1));
-    }
-    __syncthreads();
-    if (!*last_flag) return;
-    __threadfence();
+    if (!split_arrive(&p.counters[b * p.Hkv + g], static_cast<uint32_t>(p.nsplit), last_flag)) return;
     merge_split_partials<G, kTcD, Lay::kThreads>(p, b, g, ri, sb);
     if (tid == 0) p.counters[b * p.Hkv + g] = 0u;  // ready for the next step (stream-ordered)
 }
