@@ -141,6 +141,7 @@ def test_ragged_batch_limit(duo):
 @pytest.mark.parametrize("G,lens,n_tok", [
     (1, [100, 37, 260], [50, 129, 7]),   # the third sequence's second query tile is empty
     (2, [0, 300, 3], [200, 1, 130]),     # a fresh sequence, a one-token chunk, a chunk over the sinks
+    (1, [40, 0, 200], [0, 150, 129]),    # a sequence without a chunk; full and partial query tiles
 ])
 def test_ragged_prefill_then_decode(duo, G, lens, n_tok):
     Hkv = 4
