@@ -14,15 +14,11 @@
 // kernel writes, and waits for it to complete before its own CTAs exit, so the
 // pair completes as one stream-ordered step.
 //
-// Key tiles of 128 keys are listed per item and fully masked tiles are never
-// listed:
-//   retrieval: cache tiles covering [0, len) of the retrieval pool, then chunk
-//              tiles 0 .. (the diagonal tile);
-//   streaming: the streaming-cache tiles holding the sinks (and the ring when
-//              the window of the first query reaches below len), chunk tiles
-//              holding chunk-resident sinks, then the band tiles
-//              [first query - recent + 1, last query].
-// Keys are masked element-wise by absolute position only on tiles that need it.
+// Key tiles of 128 keys are listed per item (fully masked tiles never are): the
+// streaming-cache tiles holding the sinks (and the ring when the window of the
+// first query reaches below len), chunk tiles holding chunk-resident sinks, then
+// the band tiles [first query - recent + 1, last query]. Keys are masked
+// element-wise by absolute position only on tiles that need it.
 //
 // Warp roles (384 threads):
 //   warps 0-7  softmax, two threads per query row: warps w and w+4 read the
@@ -40,12 +36,13 @@
 // key half 0 at [256, 256+D) and of key half 1 at [256+D, 256+2D).
 // Key tile j (counted over the CTA's items) uses S buffer j&1, so the tensor
 // core computes S(j+1) while the softmax works on S(j). Each half writes its P
-// (bf16 pairs) back into the S buffer it read, at column +32 (keys 0-63) or +64 (keys 64-127), and the PV
-// product of that half (A operand in TMEM, four K=16 steps) accumulates into
-// its own O as soon as its four warps are done. MMA issue order per key tile j
-// (one thread; tcgen05 MMAs run in issue order, so a later QK never overwrites
-// a P before the PV that reads it): PV_0(j), PV_1(j), QK(j+2). An item's first
-// PV overwrites O, after the previous item's epilogue has read it.
+// (bf16 pairs) back into the S buffer it read, at column +32 (keys 0-63) or +64
+// (keys 64-127), and the PV product of that half (A operand in TMEM, four K=16
+// steps) accumulates into its own O as soon as its four warps are done. MMA
+// issue order per key tile j (one thread; tcgen05 MMAs run in issue order, so a
+// later QK never overwrites a P before the PV that reads it): PV_0(j), PV_1(j),
+// QK(j+2), where a QK of a new item waits for the last PV of the previous one.
+// An item's first PV overwrites O, after the previous item's epilogue has read it.
 // Softmax runs in the exp2 domain with a stale-max rule: O and the row sum are
 // rescaled only when the row max grows by more than 2^8 (exact: both stay
 // relative to the same stale max).
@@ -67,7 +64,7 @@ struct Layout {
     static constexpr int kQ = 0;
     static constexpr int kK = kQ + kTile;              // kKStages stages
     static constexpr int kV = kK + kKStages * kTile;   // 2 stages
-    static constexpr int kO = kV + 2 * kTile;    // output tile staged for the tile store
+    static constexpr int kO = kV + 2 * kTile;          // output tile staged for the tile store
     static constexpr int kBar = kO + kTile;
     // Epilogue exchange of the two halves of a row: maxima and row sums
     // [item parity][half][row].
@@ -85,8 +82,8 @@ static_assert(Layout<128>::kAlloc <= 227 * 1024, "shared memory of one CTA");
 // mbarrier indices
 constexpr int kQFull = 0;       // one phase per item
 constexpr int kQEmpty = 1;      // one phase per item: every QK of the item has run
-constexpr int kKFull = 2;       // + K stage
-constexpr int kKEmpty = 5;      // + K stage
+constexpr int kKFull = 2;       // + K stage (room for 3)
+constexpr int kKEmpty = 5;      // + K stage (room for 3)
 constexpr int kVFull = 8;       // + V stage
 constexpr int kVEmpty = 10;     // + V stage
 constexpr int kSFull = 12;      // + S buffer
@@ -189,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ work items, Q and K
         // Takes the next item of the launch (heaviest first) as soon as the K tiles
         // of the previous one are issued, publishes it to the other roles, loads its
-        // Q into the free Q buffer and then its K tiles.
+        // Q once the previous item's QKs have run, then its K tiles.
         if (lane == 0) {
             tma_prefetch_desc(&maps.q);
             // Test of the bounded waits: CTA 0 never issues its first K tile.
