@@ -337,12 +337,7 @@ def run_gpu(args):
         "metric": METRIC, "value": world * tok_per_step / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads,
-                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
-                   "retrieval_kv_heads": int(sum(step.mask)), "sink": w.sink, "recent": w.recent,
-                   "prefill_len": w.prefill_len, "chunk": w.chunk, "decode_steps": w.decode_steps,
-                   "seq_len": step.T, "global_batch": w.batch * world,
-                   "parallelism": "replicas" if world > 1 else "single", "l2": "inputs larger than L2"},
+        "config": main_config(w, step.mask, world),
         "prefill": {"unmasked_tflops": prefill_tflops, "ms": t_pf, "unmasked_flop": sum(pf),
                     "frac_of_measured_burst": prefill_tflops / peaks["bf16_tflops"],
                     "frac_of_nominal_2250": prefill_tflops / 2250.0},
@@ -547,6 +542,15 @@ def cpu_baseline(step_or_inputs, budget_s=15.0, stride=None):
                       f"positions), all {w.num_q_heads} heads, batch {w.batch}; fp64 C oracle, OpenMP"}
 
 
+def main_config(w, mask, world):
+    """The `config` of the headline line, shared by both arms."""
+    return {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "retrieval_kv_heads": int(sum(mask)), "sink": w.sink, "recent": w.recent,
+            "prefill_len": w.prefill_len, "chunk": w.chunk, "decode_steps": w.decode_steps,
+            "seq_len": w.prefill_len + w.decode_steps, "global_batch": w.batch * world,
+            "parallelism": "replicas" if world > 1 else "single", "l2": "inputs larger than L2"}
+
+
 def run_reference(args):
     world, rank, local = dist_env()
     if world > 1 and rank != 0:
@@ -572,9 +576,7 @@ def run_reference(args):
     res = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads, "head_dim": w.head_dim,
-                      "prefill_len": w.prefill_len, "chunk": w.chunk, "decode_steps": w.decode_steps,
-                      "seq_len": T, "parallelism": "single"},
+           "config": main_config(w, mask, world),
            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
                             "sample": r["sample"] + " per step"},
            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -71,3 +71,28 @@ def test_append_bytes_counts_written_slots():
         kept = [p for p in pos if p < w.sink or p >= L + n - w.recent]
         rows = n + len(kept)
         assert bench.append_bytes(w, mask, L, n) == rows * 2 * 8 * 2 * 2, (L, n)
+
+
+def test_reference_arm_line():
+    """`bench.py --impl reference` (the oracle timed on the host cores) prints one
+    line with the headline's metric, unit, direction and config, its own
+    cpu_baseline and an e2e block without host-device copies."""
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "1",
+                          "--cpu-budget", "1"], cwd=root, env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    w = workloads.LLAMA2_MHA
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "tokens/s"
+    assert d["higher_is_better"] is True and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 1
+    assert d["config"] == bench.main_config(w, workloads.retrieval_mask(w), 1)
+    assert d["value"] > 0 and d["value"] == d["cpu_baseline"]["value"] == d["e2e"]["value"]
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
