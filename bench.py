@@ -206,7 +206,11 @@ class Step:
         self.cache = duo.DuoCache(1, w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.sink, w.recent,
                                   self.T, self.mask, device=device)
         self.h = self.cache.handle
-        self.launches_per_step = 2 * self.n_chunks + w.decode_steps
+        # Per chunk: the retrieval-item prefill kernel and the streaming-item one (each
+        # only when the layer has heads of that kind), and the append; one decode per token.
+        r = int(sum(self.mask))
+        self.prefill_launches_per_chunk = int(r > 0) + int(r < len(self.mask))
+        self.launches_per_step = (self.prefill_launches_per_chunk + 1) * self.n_chunks + w.decode_steps
 
     def run(self, stream_ptr, events=None):
         """Enqueue one step. events: dict kind -> list of (start, end) to record around launches."""
@@ -310,7 +314,8 @@ def run_gpu(args):
     kernels = {
         # Every prefill launch is timed on its own (CUDA events around it): the burst peak applies.
         "prefill": {"bound": "tensor", "achieved": prefill_tflops, "peak": peaks["bf16_tflops"],
-                    "unit": "TFLOP/s", "ms_per_step": t_pf, "launches_per_step": step.n_chunks},
+                    "unit": "TFLOP/s", "ms_per_step": t_pf,
+                    "launches_per_step": step.prefill_launches_per_chunk * step.n_chunks},
         "decode": {"bound": "hbm", "achieved": decode_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                    "ms_per_step": t_dc, "launches_per_step": w.decode_steps},
         "append": {"bound": "hbm", "achieved": append_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
